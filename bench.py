@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the linear-attention hot path on B200.
+
+One step = the whole path for one batch of synthetic input: S_0 = 0, the
+chunkwise prefill of every sequence (la_prefill), then `decode_steps` decode
+tokens per sequence (la_decode_step), all through the C ABI.  Default
+workload: B=8 sequences x H=16 heads, T=8192 tokens, d_k=d_v=128, bf16
+inputs with L2-normalised keys, chunk 64, 256 decode steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): units are independent, so every rank
+runs its own batch (weak scaling, no data-path collective); the barrier and
+the max-over-ranks time use NCCL.  Rank 0 prints one JSON line.
+
+The reference arm (--impl reference) times the float64 CPU oracle (the
+literal token-by-token recurrence) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s and % of bf16 tensor peak; decode tokens/s and % HBM BW (1×B200)"
+DEFAULT_WORKLOAD = "b8h16_t8192_d128_knorm"
+L2_BYTES_FALLBACK = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--chunk", type=int, default=0, help="0 = the workload's chunk size")
+    ap.add_argument("--decode-steps", type=int, default=-1, help="-1 = the workload's count")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cold-decode", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target wall time of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- helpers --
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self.t is not None:
+                self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, p in zip(names, parts[5:9]):
+                if p.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------ algorithmic sizes --
+
+def prefill_bytes(units, T, dk, dv, elem):
+    """Q, K, V read and O written once, S_0 read and S_T written once."""
+    return units * T * (2 * dk + 2 * dv) * elem + units * 2 * dk * dv * 4
+
+
+def prefill_flops_dense(units, T, dk, dv, C):
+    """Dense-tile tensor work: QK^T (2C d_k), PV (2C d_v), QS and K^T V (2 d_k d_v each) per token."""
+    return units * T * (2 * C * dk + 2 * C * dv + 4 * dk * dv)
+
+
+def decode_bytes(units, dk, dv, elem):
+    """State read + written (fp32), q, k, v read and o written."""
+    return units * (8 * dk * dv + elem * (2 * dk + 2 * dv))
+
+
+# ----------------------------------------------------------- reference arm --
+
+def _oracle_pass(wl, units, dsteps):
+    """One pass of the whole path on `units` (sequence, head) units with the
+    float64 oracle: full prefill, then `dsteps` decode tokens.  Returns seconds
+    spent in the oracle (input generation excluded)."""
+    import numpy as np
+    from oracle import la_oracle as ora
+    from recurrent_decode_la_b200 import inputs
+    qkv = [inputs.unit_qkv(wl, u) for u in units]
+    Q = np.stack([x[0].float().numpy() for x in qkv])[:, None]
+    K = np.stack([x[1].float().numpy() for x in qkv])[:, None]
+    V = np.stack([x[2].float().numpy() for x in qkv])[:, None]
+    dec = [inputs.decode_token(wl, s, units=max(units) + 1) for s in range(dsteps)]
+    t0 = time.perf_counter()
+    _, S = ora.recurrent(Q, K, V)
+    S = S.reshape(len(units), wl.d, wl.d)
+    for dq, dk_, dv in dec:
+        _, S = ora.decode_step(dq[units], dk_[units], dv[units], S)
+    return time.perf_counter() - t0
+
+
+def _oracle_units_for(wl, seconds, dsteps):
+    """How many units make one oracle pass last about `seconds`."""
+    from oracle import la_oracle as ora
+    from recurrent_decode_la_b200 import inputs
+    cores = ora.max_threads()
+    n_units = inputs.n_units(wl)
+    probe = list(range(min(cores, n_units)))
+    t = _oracle_pass(wl, probe, wl.decode_steps and min(wl.decode_steps, dsteps))
+    per_round = max(t, 1e-3)               # one unit per core in parallel
+    rounds = max(1, int(seconds / per_round))
+    return min(n_units, rounds * len(probe)), cores
+
+
+def run_reference(args, wl, world, rank):
+    """The reference arm: the float64 CPU oracle (C recurrence over OpenMP
+    threads) timed on a bounded sample of the same workload."""
+    if rank != 0:
+        return 0
+    from recurrent_decode_la_b200 import inputs
+    dsteps = wl.decode_steps if args.decode_steps < 0 else args.decode_steps
+    n_units = inputs.n_units(wl)
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps + args.warmup))
+    units, cores = _oracle_units_for(wl, per_step, dsteps)
+    sample = list(range(units))
+    times = []
+    for it in range(args.warmup + args.steps):
+        t = _oracle_pass(wl, sample, dsteps)
+        if it >= args.warmup:
+            times.append(t)
+    tot = sum(times)
+    tokens = args.steps * units * (wl.T + dsteps) / wl.H   # a token carries H heads
+    value = tokens / tot
+    desc = (f"{units} of {n_units} (sequence, head) units per step: full T={wl.T} prefill + "
+            f"{dsteps} decode tokens each, float64 recurrence; tokens = unit rows / H")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "d_k": wl.d, "d_v": wl.d,
+                   "decode_steps": dsteps, "sample_units": units, "of_units": n_units},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline_sample(wl, seconds, dsteps):
+    """The oracle on the host cores, one bounded pass (rank 0, N=1 only)."""
+    from recurrent_decode_la_b200 import inputs
+    units, cores = _oracle_units_for(wl, seconds, dsteps)
+    t = _oracle_pass(wl, list(range(units)), dsteps)
+    tokens = units * (wl.T + dsteps) / wl.H
+    return {"value": tokens / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{units} of {inputs.n_units(wl)} (sequence, head) units: full T={wl.T} prefill + "
+                      f"{dsteps} decode tokens each, float64 recurrence, {t:.1f} s; tokens = unit rows / H"}
+
+
+# ------------------------------------------------------------------ our arm --
+
+def run_ours(args, wl, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import recurrent_decode_la_b200 as la
+    from recurrent_decode_la_b200 import inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    la.load_library()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks, peak_src = load_peaks()
+    B, H, T, d = wl.B, wl.H, wl.T, wl.d
+    chunk = args.chunk or wl.chunk
+    dsteps = wl.decode_steps if args.decode_steps < 0 else args.decode_steps
+    units = B * H
+    elem = 2 if wl.dtype == "bf16" else 4
+    dt = wl.torch_dtype
+
+    # every rank runs its own batch of the same shape (weak scaling)
+    q_h, k_h, v_h, _ = inputs.prefill_inputs(wl)
+    dq_h, dk_h, dv_h = [], [], []
+    for s in range(dsteps):
+        a, b_, c = inputs.decode_token(wl, s, units=units)
+        dq_h.append(a); dk_h.append(b_); dv_h.append(c)
+    dq_h = torch.stack(dq_h).reshape(dsteps, B, H, d) if dsteps else torch.empty(0, B, H, d, dtype=dt)
+    dk_h = torch.stack(dk_h).reshape(dsteps, B, H, d) if dsteps else torch.empty(0, B, H, d, dtype=dt)
+    dv_h = torch.stack(dv_h).reshape(dsteps, B, H, d) if dsteps else torch.empty(0, B, H, d, dtype=dt)
+
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    dq, dk_, dv = dq_h.to(dev), dk_h.to(dev), dv_h.to(dev)
+    o = torch.empty_like(v)
+    od = torch.empty_like(dv)
+    state = torch.empty(units, d, d, dtype=torch.float32, device=dev)
+    path = la.la_prefill_path(dt, d, d, chunk, q, k, v, o)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def prefill_phase(s):
+        la.la_state_init(state, None, stream=s)
+        la.la_prefill(q, k, v, o, state, chunk=chunk, stream=s)
+
+    def decode_phase(s):
+        for i in range(dsteps):
+            la.la_decode_step(dq[i], dk_[i], dv[i], od[i], state, stream=s)
+
+    # warm the launch path (sets kernel attributes) before capturing graphs
+    with torch.cuda.stream(stream):
+        prefill_phase(stream)
+        decode_phase(stream)
+    stream.synchronize()
+    if la.la_device_status(stream) != la.LA_OK:
+        raise RuntimeError("device status not ok after warm-up")
+
+    g_pre, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_pre, stream=stream):
+        prefill_phase(torch.cuda.current_stream())
+    with torch.cuda.graph(g_dec, stream=stream):
+        decode_phase(torch.cuda.current_stream())
+
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            g_pre.replay()
+            g_dec.replay()
+    stream.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            t_start.record(stream)
+            for i in range(args.steps):
+                ev[i][0].record(stream)
+                g_pre.replay()
+                ev[i][1].record(stream)
+                g_dec.replay()
+                ev[i][2].record(stream)
+            t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    status = la.la_device_status(stream)
+    ms_total = t_start.elapsed_time(t_end)
+    ms_pre = [e[0].elapsed_time(e[1]) for e in ev]
+    ms_dec = [e[1].elapsed_time(e[2]) for e in ev]
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+
+    tokens_step = B * T + B * dsteps              # sequence positions (all heads)
+    value = world * args.steps * tokens_step / (ms_total * 1e-3)
+    pre_ms = statistics.mean(ms_pre)
+    dec_ms = statistics.mean(ms_dec) if dsteps else 0.0
+    pre_bytes = prefill_bytes(units, T, d, d, elem)
+    pre_flops = prefill_flops_dense(units, T, d, d, chunk)
+    dec_bytes = decode_bytes(units, d, d, elem)
+    # prefill launch = state init + prefill kernel; the state init moves
+    # units*d*d*4 bytes and is counted in its own launch below.
+    pre_gbs = pre_bytes / (pre_ms * 1e-3) / 1e9
+    dec_us = 1e3 * dec_ms / max(1, dsteps)
+    dec_gbs = dec_bytes / (dec_us * 1e-6) / 1e9 if dsteps else 0.0
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "B": B, "H": H, "T": T, "d_k": d, "d_v": d, "chunk": chunk,
+                   "decode_steps": dsteps, "prefill_kernel": path,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (q/k/v %.0f MB per rank); decode state is the "
+                         "prefill's output and stays L2-resident within a step" % (3 * q.numel() * elem / 1e6)},
+        "prefill": {"tokens_per_s": B * T / (pre_ms * 1e-3), "ms": pre_ms,
+                    "achieved_gbs": pre_gbs, "hbm_frac": pre_gbs / peaks["hbm_gbs"],
+                    "dense_tflops": pre_flops / (pre_ms * 1e-3) / 1e12,
+                    "tensor_frac_burst": pre_flops / (pre_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                    "tensor_frac_sustained": pre_flops / (pre_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]},
+        "decode": {"tokens_per_s": B * dsteps / (dec_ms * 1e-3) if dsteps else 0.0,
+                   "us_per_step": dec_us, "achieved_gbs_l2_resident": dec_gbs},
+        "gpu_launches": args.steps * (2 + dsteps),
+        "device_status": la.la_status_string(status),
+        "peaks_source": peak_src,
+    }
+    # dominant kernel by device time within the step
+    pre_share = pre_ms / (pre_ms + dec_ms) if (pre_ms + dec_ms) > 0 else 1.0
+    roof_pre = {"bound": "hbm", "kernel": f"prefill_{path}", "achieved": pre_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": pre_gbs / peaks["hbm_gbs"], "traffic": None,
+                "bytes_per_launch": pre_bytes, "share_of_step": pre_share,
+                "peak_source": f"{peak_src} hbm_gbs"}
+    roof_dec = {"bound": "hbm", "kernel": "decode_vec", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"] if dsteps else 0.0, "traffic": None,
+                "bytes_per_launch": dec_bytes, "share_of_step": 1 - pre_share,
+                "note": "state L2-resident (stepped in place)", "peak_source": f"{peak_src} hbm_gbs"}
+    result["roofline"] = roof_pre if pre_share >= 0.5 else roof_dec
+    result["roofline_prefill"] = roof_pre
+    result["clocks"] = clk.summary()
+
+    if not args.no_cold_decode and dsteps:
+        result["decode_cold"] = cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_src)
+
+    if not args.no_e2e:
+        result["e2e"] = e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h, dk_h, dv_h,
+                                world)
+    if world > 1:
+        dist.barrier()
+    del g_pre, g_dec
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline_sample(wl, args.cpu_seconds, dsteps)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_src):
+    """Decode with a cold state: rotate over R state sets larger than L2 (as a
+    stack of R layers would), one launch per set, timed with CUDA events."""
+    d = wl.d
+    try:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    except Exception:
+        l2 = L2_BYTES_FALLBACK
+    per = units * d * d * 4
+    R = max(8, int(math.ceil(2.5 * l2 / per)))
+    states = torch.zeros(R, units, d, d, dtype=torch.float32, device=dev)
+    reps = 4
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            la.la_decode_step(dq[r % dq.shape[0]], dk_[r % dq.shape[0]], dv[r % dq.shape[0]], od[0], states[r],
+                              stream=stream)
+    stream.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            for r in range(R):
+                la.la_decode_step(dq[r % dq.shape[0]], dk_[r % dq.shape[0]], dv[r % dq.shape[0]], od[0], states[r],
+                                  stream=torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / (reps * R)
+    elem = 2 if wl.dtype == "bf16" else 4
+    byts = decode_bytes(units, d, d, elem)
+    gbs = byts / (us * 1e-6) / 1e9
+    del g, states
+    return {"us_per_launch": us, "units": units, "state_sets": R, "bytes_per_launch": byts,
+            "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
+            "tokens_per_s": wl.B / (us * 1e-6)}
+
+
+def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h, dk_h, dv_h, world):
+    """Same step through the public API with host buffers: pinned host -> device
+    copies of every input, and device -> host copies of every output, timed."""
+    B, H, T, d = wl.B, wl.H, wl.T, wl.d
+    pins = [x.pin_memory() for x in (q_h, k_h, v_h, dq_h, dk_h, dv_h)]
+    o_h = torch.empty_like(pins[2]).pin_memory()
+    od_h = torch.empty_like(pins[5]).pin_memory()
+    st_h = torch.empty(B * H, d, d, dtype=torch.float32).pin_memory()
+    dev_bufs = [torch.empty_like(x, device=dev) for x in pins]
+    o = torch.empty_like(dev_bufs[2])
+    od = torch.empty_like(dev_bufs[5])
+    st = torch.empty(B * H, d, d, dtype=torch.float32, device=dev)
+
+    def step():
+        for h, dbuf in zip(pins, dev_bufs):
+            dbuf.copy_(h, non_blocking=True)
+        la.la_state_init(st, None, stream=stream)
+        la.la_prefill(dev_bufs[0], dev_bufs[1], dev_bufs[2], o, st, chunk=chunk, stream=stream)
+        for i in range(dsteps):
+            la.la_decode_step(dev_bufs[3][i], dev_bufs[4][i], dev_bufs[5][i], od[i], st, stream=stream)
+        o_h.copy_(o, non_blocking=True)
+        od_h.copy_(od, non_blocking=True)
+        st_h.copy_(st, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            step()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    h2d = sum(x.numel() * x.element_size() for x in pins)
+    d2h = o_h.numel() * o_h.element_size() + od_h.numel() * od_h.element_size() + st_h.numel() * 4
+    tokens = B * T + B * dsteps
+    return {"value": world * args.steps * tokens / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    from recurrent_decode_la_b200 import inputs
+    wl = inputs.WORKLOADS[args.workload]
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, wl, world, rank)
+    return run_ours(args, wl, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,232 @@
+// la_api.cu -- the C ABI of liblinattn.so (declared in include/linattn.h):
+// argument checks, kernel choice, TMA descriptors and launches.  Host code
+// only; every step of the computation runs in the kernels.
+#include <cudaTypedefs.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/linattn.h"
+#include "la_device.cuh"
+#include "la_internal.h"
+
+namespace la {
+
+__device__ unsigned int g_error_word[2];
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+la_status cuda_fail(cudaError_t e) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return LA_ERR_CUDA;
+}
+
+int current_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+uint64_t wait_timeout_ns() {
+    static uint64_t v = [] {
+        const char* e = getenv("LINATTN_WAIT_TIMEOUT_MS");
+        double ms = e ? atof(e) : 4000.0;
+        if (!(ms > 0)) ms = 4000.0;
+        return static_cast<uint64_t>(ms * 1e6);
+    }();
+    return v;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 view (d, rows, groups) of a [groups][rows][d] tensor, box
+// (64, chunk, 1), 128-byte swizzle: one box fills one swizzled smem panel.
+bool encode_bf16_map(CUtensorMap* map, const void* base, int d, int64_t rows, int64_t groups, int chunk) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(groups)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(chunk), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int default_chunk(la_dtype dtype, int dk, int dv) {
+    const char* e = getenv("LINATTN_CHUNK");
+    if (e) {
+        const int c = atoi(e);
+        if (c > 0) return c;
+    }
+    if (dtype == LA_BF16 && dk == dv && (dk == 64 || dk == 128)) return 64;
+    return dk <= 32 && dv <= 32 ? 32 : 16;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+enum Path { kTc, kSimt, kUnsupported };
+
+Path choose_path(la_dtype dtype, int dk, int dv, int chunk, const void* q, const void* k, const void* v,
+                 const void* o) {
+    if (dk < 1 || dv < 1 || dk > 128 || dv > 128 || chunk < 1) return kUnsupported;
+    if (dtype == LA_BF16 && dk == dv && prefill_tc_supported(dk, chunk) && aligned16(q) && aligned16(k) &&
+        aligned16(v) && aligned16(o))
+        return kTc;
+    if (prefill_simt_smem_bytes(dk, dv, chunk) <= 227 * 1024) return kSimt;
+    return kUnsupported;
+}
+
+}  // namespace
+}  // namespace la
+
+using namespace la;
+
+extern "C" {
+
+const char* la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "ok";
+        case LA_ERR_INVALID_ARG: return "invalid argument";
+        case LA_ERR_UNSUPPORTED: return "unsupported";
+        case LA_ERR_CUDA: return "CUDA error";
+        case LA_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char* la_last_cuda_error(void) { return g_last_cuda_error; }
+
+int la_resolve_chunk(la_dtype dtype, int d_k, int d_v, int chunk) {
+    return chunk > 0 ? chunk : default_chunk(dtype, d_k, d_v);
+}
+
+const char* la_prefill_path(la_dtype dtype, int d_k, int d_v, int chunk, const void* q, const void* k,
+                            const void* v, const void* o) {
+    const int c = la_resolve_chunk(dtype, d_k, d_v, chunk);
+    switch (choose_path(dtype, d_k, d_v, c, q, k, v, o)) {
+        case kTc: return "tc";
+        case kSimt: return "simt";
+        default: return "unsupported";
+    }
+}
+
+la_status la_state_init(float* state, const float* src, int64_t n_units, int d_k, int d_v, void* stream) {
+    if (n_units < 0 || d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
+    if (n_units == 0) return LA_OK;
+    if (!state) return LA_ERR_INVALID_ARG;
+    cudaError_t e = launch_state_init(state, src, n_units * d_k * d_v, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e);
+}
+
+size_t la_prefill_workspace_size(la_dtype dtype, int B, int H, int64_t T, int d_k, int d_v, int num_seqs,
+                                 int chunk) {
+    (void)dtype; (void)B; (void)H; (void)T; (void)d_k; (void)d_v; (void)num_seqs; (void)chunk;
+    return 0;
+}
+
+la_status la_prefill(const void* q, const void* k, const void* v, void* o, float* state, la_dtype dtype, int B,
+                     int H, int64_t T, int d_k, int d_v, const int32_t* cu_seqlens, int num_seqs,
+                     int64_t max_seqlen, int chunk, void* workspace, size_t workspace_bytes, void* stream) {
+    (void)max_seqlen; (void)workspace; (void)workspace_bytes;
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || T < 0 || d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
+    if (T > 0x7fffffffLL) return LA_ERR_UNSUPPORTED;
+    int64_t n_units, groups;
+    if (cu_seqlens) {
+        if (B != 1 || num_seqs < 0) return LA_ERR_INVALID_ARG;
+        n_units = static_cast<int64_t>(num_seqs) * H;
+        groups = H;
+    } else {
+        n_units = static_cast<int64_t>(B) * H;
+        groups = n_units;
+    }
+    if (n_units == 0 || T == 0) return LA_OK;
+    if (!q || !k || !v || !o || !state) return LA_ERR_INVALID_ARG;
+    const int c = la_resolve_chunk(dtype, d_k, d_v, chunk);
+    Path path = choose_path(dtype, d_k, d_v, c, q, k, v, o);
+    if (path == kUnsupported) return LA_ERR_UNSUPPORTED;
+    // The tensor-core kernel moves state rows with 16-byte accesses.
+    if (path == kTc && !aligned16(state)) path = kSimt;
+    if (path == kSimt && prefill_simt_smem_bytes(d_k, d_v, c) > 227 * 1024) return LA_ERR_UNSUPPORTED;
+
+    PrefillProblem p;
+    p.q = q; p.k = k; p.v = v; p.o = o; p.state = state;
+    p.dtype = dtype == LA_BF16 ? 1 : 0;
+    p.H = H > 0 ? H : 1;
+    p.rows_per_group = T;
+    p.n_units = n_units;
+    p.dk = d_k; p.dv = d_v;
+    p.cu = cu_seqlens;
+    p.chunk = c;
+    p.timeout_ns = wait_timeout_ns();
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int sms = current_sm_count();
+    cudaError_t e;
+    if (path == kTc) {
+        CUtensorMap tq, tk, tv, to;
+        if (!encode_bf16_map(&tq, q, d_k, T, groups, c) || !encode_bf16_map(&tk, k, d_k, T, groups, c) ||
+            !encode_bf16_map(&tv, v, d_v, T, groups, c) || !encode_bf16_map(&to, o, d_v, T, groups, c)) {
+            snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
+            return LA_ERR_CUDA;
+        }
+        e = launch_prefill_tc(p, tq, tk, tv, to, sms, s);
+    } else {
+        e = launch_prefill_simt(p, sms, s);
+    }
+    return e == cudaSuccess ? LA_OK : cuda_fail(e);
+}
+
+la_status la_decode_step(const void* q, const void* k, const void* v, void* o, float* state, la_dtype dtype,
+                         int B, int H, int d_k, int d_v, void* stream) {
+    if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
+    if (d_k > 128 || d_v > 128) return LA_ERR_UNSUPPORTED;
+    const int64_t n_units = static_cast<int64_t>(B) * H;
+    if (n_units == 0) return LA_OK;
+    if (!q || !k || !v || !o || !state) return LA_ERR_INVALID_ARG;
+    cudaError_t e = launch_decode(q, k, v, o, state, dtype == LA_BF16 ? 1 : 0, n_units, d_k, d_v,
+                                  current_sm_count(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? LA_OK : cuda_fail(e);
+}
+
+la_status la_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned int w[2] = {0, 0};
+    e = cudaMemcpyFromSymbol(w, g_error_word, sizeof(w));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (w[0] != 0) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "device wait gave up at site 0x%x", w[1]);
+        const unsigned int z[2] = {0, 0};
+        e = cudaMemcpyToSymbol(g_error_word, z, sizeof(z));
+        if (e != cudaSuccess) return cuda_fail(e);
+        return LA_ERR_TIMEOUT;
+    }
+    return LA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,607 @@
+// la_prefill_tc.cu -- chunkwise causal linear-attention prefill on the B200
+// tensor cores (sm_100a: TMA + tcgen05 + TMEM).
+//
+// The computation is the chunkwise form of the slides "Chunking, causality,
+// and parallel prefill" (sections "Split into chunks", "Causal triangle",
+// "Incoming and outgoing state"): for every chunk c of C tokens of a unit,
+//     A   = Q_c K_c^T                      (C x C, fp32 in TMEM)
+//     P   = A with j > i set to 0          (diagonal kept; bf16 in smem)
+//     O_c = Q_c S_{c-1} + P V_c            (one fp32 TMEM accumulator)
+//     S_c = S_{c-1} + K_c^T V_c            (fp32 in TMEM for the whole unit)
+// The only serial hop between chunks is S: after K_c^T V_c lands in TMEM,
+// the state is copied out once as a bf16 operand for the next chunk's Q S.
+//
+// One persistent CTA per SM walks units (one sequence of one head) with a
+// static stride.  Warp roles (384 threads):
+//   warp 0      TMA producer: Q/K/V chunk tiles into an NS-deep ring
+//   warp 1      MMA issuer (one thread) and TMEM owner
+//   warps 4-7   "state" warpgroup: causal mask -> P, state hop S -> bf16,
+//               S_0 in and S_T out
+//   warps 8-11  "output" warpgroup: O TMEM -> bf16 -> smem -> TMA store
+// Every wait is an mbarrier wait bounded by a timeout; on expiry the kernel
+// records the error word, every role winds down, outstanding copies and
+// MMAs are drained (bounded), TMEM is freed and the kernel returns.
+#include "la_device.cuh"
+#include "la_internal.h"
+
+namespace la {
+
+template <int C, int D>
+struct TcCfg {
+    static constexpr int kThreads = 384;
+    static constexpr int PANEL = C * 128;  // one 64-column panel of a chunk tile (bytes)
+    static constexpr int NPAN = D / 64;
+    static constexpr int TILE = C * D * 2;
+    static constexpr int STAGE = 3 * TILE;  // Q, K, V of one chunk
+    static constexpr int NS = (C == 64 && D == 64) ? 6 : (C == 64 ? 3 : (D == 64 ? 2 : 1));
+    static constexpr int PB = 2;                           // P buffers
+    static constexpr int OB = (C == 128 && D == 128) ? 1 : 2;  // O accumulators in TMEM
+    static constexpr int OSB = (C == 128 && D == 128) ? 1 : 2;  // O staging buffers
+    static constexpr int P_BYTES = C * C * 2;
+    static constexpr int P_PANEL = C * 128;
+    static constexpr int SB_BYTES = D * D * 2;
+    static constexpr int SB_PANEL = D * 128;
+    static constexpr int OST_BYTES = C * D * 2;
+    static constexpr int OFF_STAGE = 0;
+    static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
+    static constexpr int OFF_SB = OFF_P + PB * P_BYTES;
+    static constexpr int OFF_OST = OFF_SB + SB_BYTES;
+    static constexpr int OFF_BAR = OFF_OST + OSB * OST_BYTES;
+    static constexpr int NBAR = 40;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
+    // tensor memory columns (fp32, 128 lanes)
+    static constexpr int TM_S = 0;
+    static constexpr int TM_O = D;
+    static constexpr int TM_A = D + OB * D;
+    static constexpr int TM_COLS = 512;
+    static_assert(TM_A + 2 * C <= TM_COLS, "tensor memory budget");
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(NS <= 6, "barrier slots");
+    // mbarrier slots
+    static constexpr int B_FULL = 0;       // [NS] TMA landed
+    static constexpr int B_EMPTY = 8;      // [NS] MMAs of the stage done
+    static constexpr int B_AFULL = 16;     // [2] scores in TMEM
+    static constexpr int B_AEMPTY = 18;    // [2] scores read out
+    static constexpr int B_PFULL = 20;     // [2] P written
+    static constexpr int B_PEMPTY = 22;    // [2] P consumed
+    static constexpr int B_SFULL = 24;     // state accumulated
+    static constexpr int B_SREAD = 25;     // state read out (may accumulate again)
+    static constexpr int B_SBFULL = 26;    // bf16 state operand written
+    static constexpr int B_SBEMPTY = 27;   // bf16 state operand consumed
+    static constexpr int B_OFULL = 28;     // [2] O accumulated
+    static constexpr int B_OEMPTY = 30;    // [2] O read out
+    static constexpr int B_OSTFULL = 32;   // [2] O staging written
+    static constexpr int B_OSTFREE = 34;   // [2] O staging read by the TMA store
+    static constexpr int B_MMADONE = 36;   // drain at teardown
+};
+
+struct Unit {
+    int group;
+    int row0;
+    int len;
+};
+
+// Rows of unit u.  A packed sequence whose offsets are out of range or
+// decreasing is treated as empty (its state is left untouched).
+__device__ __forceinline__ Unit get_unit(const PrefillProblem& p, int64_t u) {
+    if (p.cu == nullptr) return {static_cast<int>(u), 0, static_cast<int>(p.rows_per_group)};
+    const int n = static_cast<int>(u / p.H);
+    const int h = static_cast<int>(u % p.H);
+    const int a = p.cu[n];
+    const int b = p.cu[n + 1];
+    if (a < 0 || b < a || static_cast<int64_t>(b) > p.rows_per_group) return {h, 0, 0};
+    return {h, a, b - a};
+}
+
+// Accumulator row held by lane `lane` of a warp reading its TMEM
+// sub-partition `sub` with the 32x32b shape.  M = 128: row = lane index in
+// TMEM.  M = 64: rows 16*sub .. 16*sub+15 sit in lanes 0..15 of the
+// sub-partition; lanes 16..31 hold no row (-1).
+template <int M>
+__device__ __forceinline__ int acc_row(int sub, int lane) {
+    if (M == 128) return sub * 32 + lane;
+    return lane < 16 ? sub * 16 + lane : -1;
+}
+
+template <int C, int D>
+__global__ void __launch_bounds__(384, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmO, const PrefillProblem p) {
+    using Cfg = TcCfg<C, D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::NS; ++s) {
+            mbar_init(&bar[Cfg::B_FULL + s], 1);
+            mbar_init(&bar[Cfg::B_EMPTY + s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar[Cfg::B_AFULL + b], 1);
+            mbar_init(&bar[Cfg::B_AEMPTY + b], 4);
+            mbar_init(&bar[Cfg::B_PFULL + b], 4);
+            mbar_init(&bar[Cfg::B_PEMPTY + b], 1);
+            mbar_init(&bar[Cfg::B_OFULL + b], 1);
+            mbar_init(&bar[Cfg::B_OEMPTY + b], 4);
+            mbar_init(&bar[Cfg::B_OSTFULL + b], 4);
+            mbar_init(&bar[Cfg::B_OSTFREE + b], 1);
+        }
+        mbar_init(&bar[Cfg::B_SFULL], 1);
+        mbar_init(&bar[Cfg::B_SREAD], 4);
+        mbar_init(&bar[Cfg::B_SBFULL], 4);
+        mbar_init(&bar[Cfg::B_SBEMPTY], 1);
+        mbar_init(&bar[Cfg::B_MMADONE], 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base_slot, Cfg::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_slot;
+
+    const uint32_t sbase = smem_u32(smem);
+    auto stage_q = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE; };
+    auto stage_k = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + Cfg::TILE; };
+    auto stage_v = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + 2 * Cfg::TILE; };
+    const uint32_t p_base = sbase + Cfg::OFF_P;
+    const uint32_t sb_base = sbase + Cfg::OFF_SB;
+    const uint32_t ost_base = sbase + Cfg::OFF_OST;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int64_t g = 0;
+            int64_t last_g[Cfg::NS];
+            for (int s = 0; s < Cfg::NS; ++s) last_g[s] = -1;
+            bool ok = true;
+            for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+                const Unit un = get_unit(p, u);
+                const int nch = (un.len + C - 1) / C;
+                for (int c = 0; c < nch; ++c, ++g) {
+                    const int s = static_cast<int>(g % Cfg::NS);
+                    if (g >= Cfg::NS) {
+                        if (!mbar_wait(&bar[Cfg::B_EMPTY + s], ((g / Cfg::NS) + 1) & 1, abort_flag,
+                                       tmo, 0x100 + s)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    mbar_arrive_expect_tx(&bar[Cfg::B_FULL + s], Cfg::STAGE);
+                    const int row = un.row0 + c * C;
+#pragma unroll
+                    for (int pn = 0; pn < Cfg::NPAN; ++pn) {
+                        tma_load_3d(reinterpret_cast<void*>(smem + (stage_q(s) - sbase) + pn * Cfg::PANEL),
+                                    &tmQ, &bar[Cfg::B_FULL + s], pn * 64, row, un.group);
+                        tma_load_3d(reinterpret_cast<void*>(smem + (stage_k(s) - sbase) + pn * Cfg::PANEL),
+                                    &tmK, &bar[Cfg::B_FULL + s], pn * 64, row, un.group);
+                        tma_load_3d(reinterpret_cast<void*>(smem + (stage_v(s) - sbase) + pn * Cfg::PANEL),
+                                    &tmV, &bar[Cfg::B_FULL + s], pn * 64, row, un.group);
+                    }
+                    last_g[s] = g;
+                }
+            }
+            if (!ok || *abort_flag) {
+                // Let every copy this thread started land before the CTA exits.
+                for (int s = 0; s < Cfg::NS; ++s)
+                    if (last_g[s] >= 0)
+                        mbar_wait_drain(&bar[Cfg::B_FULL + s], (last_g[s] / Cfg::NS) & 1, tmo);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        constexpr uint32_t kIdQK = idesc_bf16_f32(C, C, false, false);
+        constexpr uint32_t kIdKV = idesc_bf16_f32(D, D, true, true);
+        constexpr uint32_t kIdQS = idesc_bf16_f32(C, D, false, true);
+        constexpr uint32_t kIdPV = idesc_bf16_f32(C, D, false, true);
+        const uint32_t tm_S = tmem + Cfg::TM_S;
+        int64_t g = 0;
+        bool ok = true;
+        bool issued_any = false;
+        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            const Unit un = get_unit(p, u);
+            const int nch = (un.len + C - 1) / C;
+            for (int c = 0; c < nch; ++c, ++g) {
+                const int s = static_cast<int>(g % Cfg::NS);
+                const int nv = min(C, un.len - c * C);
+                if (!mbar_wait_warp(&bar[Cfg::B_FULL + s], (g / Cfg::NS) & 1, abort_flag, tmo,
+                                    0x200 + s)) {
+                    ok = false;
+                    break;
+                }
+                if (nv < C) {
+                    // Rows past the end of the sequence must not reach the
+                    // state: zero them in the K and V tiles.
+                    const int nrow = C - nv;
+                    const int per_tile = nrow * Cfg::NPAN * 8;  // 16-byte pieces
+                    for (int i = lane; i < 2 * per_tile; i += 32) {
+                        const int t = i / per_tile;
+                        const int r = i % per_tile;
+                        const int row = nv + r / (Cfg::NPAN * 8);
+                        const int pn = (r / 8) % Cfg::NPAN;
+                        const int ch = r % 8;
+                        const uint32_t base = t == 0 ? stage_k(s) : stage_v(s);
+                        st_shared_v4(base + pn * Cfg::PANEL + row * 128 + ch * 16, 0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    const int b = static_cast<int>(g & 1);
+                    const int ob = static_cast<int>(g % Cfg::OB);
+                    const uint32_t qb = stage_q(s), kb = stage_k(s), vb = stage_v(s);
+                    // (1) A = Q K^T
+                    if (g >= 2 && !mbar_wait(&bar[Cfg::B_AEMPTY + b], ((g >> 1) + 1) & 1,
+                                             abort_flag, tmo, 0x210 + b)) {
+                        ok = false;
+                    }
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t tm_A = tmem + Cfg::TM_A + b * C;
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * Cfg::PANEL + (ks & 3) * 32;
+                            mma_bf16_ss(tm_A, sdesc_sw128(qb + off, 16, 1024),
+                                        sdesc_sw128(kb + off, 16, 1024), kIdQK, ks > 0);
+                        }
+                        mma_commit(&bar[Cfg::B_AFULL + b]);
+                        issued_any = true;
+                    }
+                    // (2) S += K^T V
+                    if (ok && !mbar_wait(&bar[Cfg::B_SREAD], g & 1, abort_flag, tmo, 0x220))
+                        ok = false;
+                    if (ok) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < C / 16; ++ks) {
+                            mma_bf16_ss(tm_S, sdesc_sw128(kb + ks * 2048, Cfg::PANEL, 1024),
+                                        sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024), kIdKV, 1);
+                        }
+                        mma_commit(&bar[Cfg::B_SFULL]);
+                    }
+                    // (3) O = Q S_prev
+                    if (ok && g >= Cfg::OB &&
+                        !mbar_wait(&bar[Cfg::B_OEMPTY + ob], ((g / Cfg::OB) + 1) & 1, abort_flag,
+                                   tmo, 0x230 + ob))
+                        ok = false;
+                    if (ok && !mbar_wait(&bar[Cfg::B_SBFULL], g & 1, abort_flag, tmo, 0x240))
+                        ok = false;
+                    const uint32_t tm_O = tmem + Cfg::TM_O + ob * D;
+                    if (ok) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * Cfg::PANEL + (ks & 3) * 32;
+                            mma_bf16_ss(tm_O, sdesc_sw128(qb + off, 16, 1024),
+                                        sdesc_sw128(sb_base + ks * 2048, Cfg::SB_PANEL, 1024),
+                                        kIdQS, ks > 0);
+                        }
+                        mma_commit(&bar[Cfg::B_SBEMPTY]);
+                    }
+                    // (4) O += P V
+                    if (ok && !mbar_wait(&bar[Cfg::B_PFULL + b], (g >> 1) & 1, abort_flag, tmo,
+                                         0x250 + b))
+                        ok = false;
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t pb = p_base + b * Cfg::P_BYTES;
+#pragma unroll
+                        for (int ks = 0; ks < C / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * Cfg::P_PANEL + (ks & 3) * 32;
+                            mma_bf16_ss(tm_O, sdesc_sw128(pb + off, 16, 1024),
+                                        sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024), kIdPV, 1);
+                        }
+                        mma_commit(&bar[Cfg::B_PEMPTY + b]);
+                        mma_commit(&bar[Cfg::B_OFULL + ob]);
+                        mma_commit(&bar[Cfg::B_EMPTY + s]);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+            }
+        }
+        if (lane == 0 && issued_any) {
+            // Drain: every MMA issued above has completed before TMEM is freed.
+            mma_commit(&bar[Cfg::B_MMADONE]);
+            mbar_wait_drain(&bar[Cfg::B_MMADONE], 0, tmo);
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------- state / mask warpgroup
+        const int sub = warp & 3;
+        const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+        const int rowA = acc_row<C>(sub, lane);  // score / P row
+        const int rowS = acc_row<D>(sub, lane);  // state row (key index)
+        const uint32_t tm_S = tmem + Cfg::TM_S + lane_off;
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            const Unit un = get_unit(p, u);
+            const int nch = (un.len + C - 1) / C;
+            if (nch == 0) continue;
+            float* st_row = p.state + u * static_cast<int64_t>(D) * D +
+                            static_cast<int64_t>(rowS < 0 ? 0 : rowS) * D;
+            // ---- unit start: S_0 into TMEM (fp32) and into the bf16 operand
+            if (g > 0 && !mbar_wait_warp(&bar[Cfg::B_SBEMPTY], (g - 1) & 1, abort_flag, tmo, 0x300)) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int cb = 0; cb < D / 32; ++cb) {
+                uint32_t r[32];
+                if (rowS >= 0) {
+                    const float4* src = reinterpret_cast<const float4*>(st_row + cb * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 f = src[i];
+                        r[4 * i + 0] = __float_as_uint(f.x);
+                        r[4 * i + 1] = __float_as_uint(f.y);
+                        r[4 * i + 2] = __float_as_uint(f.z);
+                        r[4 * i + 3] = __float_as_uint(f.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = 0u;
+                }
+                tmem_st32(tm_S + cb * 32, r);
+                if (rowS >= 0) {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int col = cb * 32 + ch * 8;  // 8 bf16 = one 16-byte chunk
+                        const uint32_t addr = sb_base + (col >> 6) * Cfg::SB_PANEL +
+                                              sw128_off(rowS, (col & 63) >> 3);
+                        st_shared_v4(addr,
+                                     pack_bf16x2(__uint_as_float(r[ch * 8 + 0]), __uint_as_float(r[ch * 8 + 1])),
+                                     pack_bf16x2(__uint_as_float(r[ch * 8 + 2]), __uint_as_float(r[ch * 8 + 3])),
+                                     pack_bf16x2(__uint_as_float(r[ch * 8 + 4]), __uint_as_float(r[ch * 8 + 5])),
+                                     pack_bf16x2(__uint_as_float(r[ch * 8 + 6]), __uint_as_float(r[ch * 8 + 7])));
+                    }
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar[Cfg::B_SREAD]);
+                mbar_arrive(&bar[Cfg::B_SBFULL]);
+            }
+            // ---- chunk loop
+            for (int c = 0; c < nch; ++c, ++g) {
+                const bool last = (c == nch - 1);
+                const int b = static_cast<int>(g & 1);
+                // P = mask(A)
+                if (!mbar_wait_warp(&bar[Cfg::B_AFULL + b], (g >> 1) & 1, abort_flag, tmo, 0x310 + b)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (g >= 2 && !mbar_wait_warp(&bar[Cfg::B_PEMPTY + b], ((g >> 1) + 1) & 1, abort_flag,
+                                              tmo, 0x320 + b)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t tm_A = tmem + Cfg::TM_A + b * C + lane_off;
+                const uint32_t pb = p_base + b * Cfg::P_BYTES;
+#pragma unroll
+                for (int cb = 0; cb < C / 32; ++cb) {
+                    uint32_t r[32];
+                    tmem_ld32(tm_A + cb * 32, r);
+                    tmem_wait_ld();
+                    if (rowA >= 0) {
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = cb * 32 + ch * 8 + 2 * e;
+                                const float a0 = (j <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e]) : 0.f;
+                                const float a1 = (j + 1 <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e + 1]) : 0.f;
+                                w[e] = pack_bf16x2(a0, a1);
+                            }
+                            const int col = cb * 32 + ch * 8;
+                            st_shared_v4(pb + (col >> 6) * Cfg::P_PANEL + sw128_off(rowA, (col & 63) >> 3),
+                                         w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bar[Cfg::B_AEMPTY + b]);
+                    mbar_arrive(&bar[Cfg::B_PFULL + b]);
+                }
+                // state hop: S_c out of TMEM
+                if (!mbar_wait_warp(&bar[Cfg::B_SFULL], g & 1, abort_flag, tmo, 0x330)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t pk[D / 2];
+#pragma unroll
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    uint32_t r[32];
+                    tmem_ld32(tm_S + cb * 32, r);
+                    tmem_wait_ld();
+                    if (last && rowS >= 0) {
+                        float4* dst = reinterpret_cast<float4*>(st_row + cb * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                 __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[cb * 16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                }
+                tc_fence_before();
+                if (!last) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar[Cfg::B_SREAD]);
+                    if (!mbar_wait_warp(&bar[Cfg::B_SBEMPTY], g & 1, abort_flag, tmo, 0x340)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rowS >= 0) {
+#pragma unroll
+                        for (int ch = 0; ch < D / 8; ++ch) {
+                            const int col = ch * 8;
+                            st_shared_v4(sb_base + (col >> 6) * Cfg::SB_PANEL + sw128_off(rowS, (col & 63) >> 3),
+                                         pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar[Cfg::B_SBFULL]);
+                }
+            }
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------- output warpgroup
+        const int sub = warp & 3;
+        const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+        const int row = acc_row<C>(sub, lane);
+        const bool elected = (warp == 8 && lane == 0);
+        uint16_t* obase = static_cast<uint16_t*>(p.o);
+        int64_t g = 0, f = 0;
+        bool ok = true;
+        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            const Unit un = get_unit(p, u);
+            const int nch = (un.len + C - 1) / C;
+            for (int c = 0; c < nch; ++c, ++g) {
+                const int ob = static_cast<int>(g % Cfg::OB);
+                const int nv = min(C, un.len - c * C);
+                if (!mbar_wait_warp(&bar[Cfg::B_OFULL + ob], (g / Cfg::OB) & 1, abort_flag, tmo,
+                                    0x400 + ob)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t pk[D / 2];
+                const uint32_t tm_O = tmem + Cfg::TM_O + ob * D + lane_off;
+#pragma unroll
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    uint32_t r[32];
+                    tmem_ld32(tm_O + cb * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[cb * 16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[Cfg::B_OEMPTY + ob]);
+                const int64_t grow0 = static_cast<int64_t>(un.group) * p.rows_per_group + un.row0 + c * C;
+                if (nv == C) {
+                    const int osb = static_cast<int>(f % Cfg::OSB);
+                    if (f >= Cfg::OSB && !mbar_wait_warp(&bar[Cfg::B_OSTFREE + osb], ((f / Cfg::OSB) + 1) & 1,
+                                                         abort_flag, tmo, 0x410 + osb)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t stg = ost_base + osb * Cfg::OST_BYTES;
+                    if (row >= 0) {
+#pragma unroll
+                        for (int ch = 0; ch < D / 8; ++ch) {
+                            const int col = ch * 8;
+                            st_shared_v4(stg + (col >> 6) * Cfg::PANEL + sw128_off(row, (col & 63) >> 3),
+                                         pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar[Cfg::B_OSTFULL + osb]);
+                    if (elected) {
+                        if (mbar_wait(&bar[Cfg::B_OSTFULL + osb], (f / Cfg::OSB) & 1, abort_flag, tmo,
+                                      0x420 + osb)) {
+#pragma unroll
+                            for (int pn = 0; pn < Cfg::NPAN; ++pn)
+                                tma_store_3d(&tmO, smem + (stg - sbase) + pn * Cfg::PANEL, pn * 64,
+                                             un.row0 + c * C, un.group);
+                            bulk_commit_group();
+                            bulk_wait_group_read<Cfg::OSB - 1>();
+                            if (f - (Cfg::OSB - 1) >= 0)
+                                mbar_arrive(&bar[Cfg::B_OSTFREE + ((f - (Cfg::OSB - 1)) % Cfg::OSB)]);
+                        }
+                    }
+                    ++f;
+                } else if (row >= 0 && row < nv) {
+                    // Last, partial chunk of a sequence: plain stores of the
+                    // valid rows only (the next sequence's rows follow).
+                    uint4* dst = reinterpret_cast<uint4*>(obase + (grow0 + row) * D);
+#pragma unroll
+                    for (int ch = 0; ch < D / 8; ++ch)
+                        dst[ch] = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+                }
+            }
+        }
+        if (elected) bulk_wait_group<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::TM_COLS);
+    }
+}
+
+bool prefill_tc_supported(int D, int chunk) {
+    return (D == 64 || D == 128) && (chunk == 64 || chunk == 128);
+}
+
+template <int C, int D>
+static cudaError_t launch_tc_impl(const PrefillProblem& p, const CUtensorMap& tq,
+                                  const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const CUtensorMap& to, int num_sms, cudaStream_t s) {
+    using Cfg = TcCfg<C, D>;
+    auto kern = prefill_tc_kernel<C, D>;
+    // Raise the dynamic shared-memory limit once per device (not inside a
+    // stream capture: the first launch on a device sets it).
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    int64_t grid = p.n_units < num_sms ? p.n_units : num_sms;
+    if (grid < 1) return cudaSuccess;
+    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::SMEM, s>>>(tq, tk, tv, to, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_tc(const PrefillProblem& p, const CUtensorMap& tq,
+                              const CUtensorMap& tk, const CUtensorMap& tv,
+                              const CUtensorMap& to, int num_sms, cudaStream_t s) {
+    if (p.dk == 64 && p.chunk == 64) return launch_tc_impl<64, 64>(p, tq, tk, tv, to, num_sms, s);
+    if (p.dk == 128 && p.chunk == 64) return launch_tc_impl<64, 128>(p, tq, tk, tv, to, num_sms, s);
+    if (p.dk == 64 && p.chunk == 128) return launch_tc_impl<128, 64>(p, tq, tk, tv, to, num_sms, s);
+    if (p.dk == 128 && p.chunk == 128) return launch_tc_impl<128, 128>(p, tq, tk, tv, to, num_sms, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace la

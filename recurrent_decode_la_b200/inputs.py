@@ -20,8 +20,11 @@ Tensor ids: 0 = q, 1 = k, 2 = v, 3 = initial state, 10/11/12 = decode q/k/v.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import functools
 import math
+import os
 from typing import Optional
 
 import numpy as np
@@ -116,6 +119,11 @@ def cu_seqlens(wl: Workload) -> torch.Tensor:
     return cu.to(torch.int32)
 
 
+@functools.lru_cache(maxsize=16)
+def _cu_cached(wl: Workload) -> torch.Tensor:
+    return cu_seqlens(wl)
+
+
 def total_tokens(wl: Workload) -> int:
     return int(cu_seqlens(wl)[-1]) if wl.varlen else wl.T
 
@@ -132,7 +140,7 @@ def unit_rows(wl: Workload, unit: int) -> tuple[int, int, int]:
     """
     if not wl.varlen:
         return unit, 0, wl.T
-    cu = cu_seqlens(wl)
+    cu = _cu_cached(wl)
     n, h = divmod(unit, wl.H)
     return h, int(cu[n]), int(cu[n + 1] - cu[n])
 
@@ -154,22 +162,23 @@ def prefill_inputs(wl: Workload, dtype: Optional[torch.dtype] = None):
     d = wl.d
     if not wl.varlen:
         shape = (wl.B, wl.H, wl.T, d)
-        q = torch.empty(shape, dtype=dt)
-        k = torch.empty(shape, dtype=dt)
-        v = torch.empty(shape, dtype=dt)
-        for u in range(wl.B * wl.H):
-            b, h = divmod(u, wl.H)
-            q[b, h], k[b, h], v[b, h] = unit_qkv(wl, u, dt)
-        return q, k, v, None
-    cu = cu_seqlens(wl)
-    Ttot = int(cu[-1])
-    shape = (1, wl.H, Ttot, d)
+        cu = None
+    else:
+        cu = cu_seqlens(wl)
+        shape = (1, wl.H, int(cu[-1]), d)
     q = torch.empty(shape, dtype=dt)
     k = torch.empty(shape, dtype=dt)
     v = torch.empty(shape, dtype=dt)
-    for u in range(wl.num_seqs * wl.H):
-        h, r0, L = unit_rows(wl, u)
-        q[0, h, r0:r0 + L], k[0, h, r0:r0 + L], v[0, h, r0:r0 + L] = unit_qkv(wl, u, dt)
+    qf, kf, vf = (x.view(-1, shape[2], d) for x in (q, k, v))
+
+    def fill(u: int) -> None:
+        g, r0, L = unit_rows(wl, u)
+        qf[g, r0:r0 + L], kf[g, r0:r0 + L], vf[g, r0:r0 + L] = unit_qkv(wl, u, dt)
+
+    # The generators release the GIL while drawing, so units fill in parallel;
+    # every unit has its own stream, so the result does not depend on order.
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(n_units(wl))))
     return q, k, v, cu
 
 

@@ -1,0 +1,262 @@
+"""Parity of the CUDA path (called through the C ABI) with the float64 oracle.
+
+Bars: bit-exact on the slides' integer trace; max |gpu - oracle| / max |oracle|
+<= 1e-4 for fp32 inputs and <= 2e-2 for bf16 inputs (fp32 accumulation), for
+the prefill output O, the decode outputs o and the final state S.
+"""
+import numpy as np
+import pytest
+import torch
+
+import recurrent_decode_la_b200 as la
+from oracle import la_oracle as ora
+from recurrent_decode_la_b200 import inputs
+from gpu_util import BF16_TOL, F32_TOL, gpu_prefill, nerr, oracle_units
+
+pytestmark = pytest.mark.gpu
+
+WL = inputs.WORKLOADS
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    la.load_library()
+    yield
+    torch.cuda.synchronize()
+    assert la.la_device_status() == la.LA_OK
+
+
+def _example_tensors(golden, dtype):
+    k = torch.tensor(golden["k"], dtype=torch.float32)
+    v = torch.tensor(golden["v"], dtype=torch.float32)
+    return (k.clone()[None, None].to(dtype), k[None, None].to(dtype), v[None, None].to(dtype))
+
+
+# ----------------------------------------------------- the slides' trace ----
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("chunk", [1, 2, 4, 8])
+def test_worked_example_bit_exact(golden, dtype, chunk):
+    q, k, v = _example_tensors(golden, dtype)
+    o, S = gpu_prefill(q, k, v, chunk=chunk)
+    assert torch.equal(o.float().cpu()[0, 0], torch.tensor(golden["chunk4"]["o"], dtype=torch.float32))
+    assert torch.equal(S.cpu()[0], torch.tensor(golden["chunk4"]["S8"], dtype=torch.float32))
+
+
+def test_worked_example_handoffs_c2(golden):
+    """Prefill the first 2, 4, 6 tokens: the states handed off are S_2, S_4, S_6."""
+    q, k, v = _example_tensors(golden, torch.float32)
+    for n, key in ((2, "S2"), (4, "S4"), (6, "S6")):
+        _, S = gpu_prefill(q[:, :, :n], k[:, :, :n], v[:, :, :n], chunk=2)
+        assert torch.equal(S.cpu()[0], torch.tensor(golden["chunk2"]["handoffs"][key], dtype=torch.float32))
+
+
+def test_worked_example_decode_bit_exact(golden):
+    """Token-by-token decode of the trace reproduces every o_t and S_8."""
+    q, k, v = _example_tensors(golden, torch.float32)
+    st = torch.zeros(1, 2, 2, device="cuda")
+    outs = []
+    for t in range(8):
+        o = torch.empty(1, 1, 2, device="cuda")
+        la.la_decode_step(q[0, :, t].cuda()[None], k[0, :, t].cuda()[None], v[0, :, t].cuda()[None], o, st)
+        outs.append(o.cpu()[0, 0])
+    assert torch.equal(torch.stack(outs), torch.tensor(golden["chunk4"]["o"], dtype=torch.float32))
+    assert torch.equal(st.cpu()[0], torch.tensor(golden["chunk4"]["S8"], dtype=torch.float32))
+
+
+# ------------------------------------------------ tiny fp32 workload ----
+
+def test_tiny_f32_prefill_and_decode():
+    wl = WL["tiny_f32_b1h1_t64_d16"]
+    q, k, v, _ = inputs.prefill_inputs(wl)
+    O_ref, S_ref = ora.recurrent(q, k, v)
+    o, S = gpu_prefill(q, k, v, chunk=wl.chunk)
+    assert nerr(o, O_ref) <= F32_TOL
+    assert nerr(S.reshape(S_ref.shape), S_ref) <= F32_TOL
+    Sd = S.clone()
+    Sr = S_ref.reshape(1, 16, 16)
+    for step in range(wl.decode_steps):
+        dq, dk_, dv = inputs.decode_token(wl, step, units=1)
+        od = torch.empty(1, 1, 16, device="cuda")
+        la.la_decode_step(dq.cuda()[None], dk_.cuda()[None], dv.cuda()[None], od, Sd)
+        o_ref, Sr = ora.decode_step(dq, dk_, dv, Sr)
+        assert nerr(od[0], o_ref) <= F32_TOL
+    assert nerr(Sd, Sr) <= F32_TOL
+
+
+# ------------------------------------- tensor-core path, several tiles ----
+
+@pytest.mark.parametrize("d,chunk", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("T", [1, 63, 64, 333])
+def test_tc_prefill_random_state(d, chunk, T):
+    assert la.la_prefill_path(torch.bfloat16, d, d, chunk) == "tc"
+    B, H = 2, 3
+    q, k, v = inputs.random_qkv(7 * T + d + chunk, B, H, T, d, d, dtype=torch.bfloat16)
+    S0 = torch.from_numpy(np.random.default_rng(T).standard_normal((B, H, d, d)).astype(np.float32)) * 0.05
+    O_ref, S_ref = ora.recurrent(q, k, v, S0)
+    o, S = gpu_prefill(q, k, v, S0=S0, chunk=chunk)
+    assert nerr(o, O_ref) <= BF16_TOL
+    assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
+
+
+def test_tc_vs_simt_same_inputs():
+    """Two kernels, two chunk sizes, one result (chunking never changes it)."""
+    q, k, v = inputs.random_qkv(3, 1, 4, 200, 64, 64, dtype=torch.bfloat16)
+    O_ref, S_ref = ora.recurrent(q, k, v)
+    res = {}
+    for chunk in (16, 32, 64, 128):
+        o, S = gpu_prefill(q, k, v, chunk=chunk)
+        res[chunk] = (o, S)
+        assert nerr(o, O_ref) <= BF16_TOL, chunk
+        assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL, chunk
+    assert la.la_prefill_path(torch.bfloat16, 64, 64, 16) == "simt"
+    assert la.la_prefill_path(torch.bfloat16, 64, 64, 64) == "tc"
+
+
+def test_misaligned_bf16_runs_simt_and_matches():
+    B, H, T, d = 1, 2, 100, 64
+    q, k, v = inputs.random_qkv(5, B, H, T, d, d, dtype=torch.bfloat16)
+    O_ref, S_ref = ora.recurrent(q, k, v)
+    buf = torch.empty(3 * q.numel() + 1, dtype=torch.bfloat16, device="cuda")
+    qd = buf[1:1 + q.numel()].view_as(q)
+    kd = buf[1 + q.numel():1 + 2 * q.numel()].view_as(q)
+    vd = buf[1 + 2 * q.numel():].view_as(q)
+    qd.copy_(q.cuda()); kd.copy_(k.cuda()); vd.copy_(v.cuda())
+    assert la.la_prefill_path(torch.bfloat16, d, d, 64, qd, kd, vd, qd) == "simt"
+    o = torch.empty(B, H, T, d, dtype=torch.bfloat16, device="cuda")
+    S = torch.zeros(B * H, d, d, device="cuda")
+    la.la_prefill(qd, kd, vd, o, S, chunk=64)
+    assert la.la_device_status() == la.LA_OK
+    assert nerr(o, O_ref) <= BF16_TOL
+    assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
+
+
+# ----------------------------------------------------- edge cases ----
+
+def test_empty_and_degenerate():
+    d = 64
+    S0 = torch.randn(2, d, d, device="cuda")
+    st = S0.clone()
+    z = torch.empty(1, 2, 0, d, dtype=torch.bfloat16, device="cuda")
+    la.la_prefill(z, z, z, z.clone(), st, chunk=64)          # T = 0: no-op
+    assert torch.equal(st, S0)
+    with pytest.raises(la.LinAttnError) as e:                  # d above 128
+        big = torch.zeros(1, 1, 4, 256, dtype=torch.bfloat16, device="cuda")
+        la.la_prefill(big, big, big, big.clone(), torch.zeros(1, 256, 256, device="cuda"))
+    assert e.value.status == la.LA_ERR_UNSUPPORTED
+    lib = la.load_library()
+    assert lib.la_prefill(None, None, None, None, None, 1, 1, 1, 8, 64, 64, None, 0, 0, 64, None, 0, None) \
+        == la.LA_ERR_INVALID_ARG
+    assert lib.la_decode_step(None, None, None, None, None, 1, 1, 1, 64, 64, None) == la.LA_ERR_INVALID_ARG
+    assert lib.la_prefill(None, None, None, None, None, 7, 1, 1, 8, 64, 64, None, 0, 0, 64, None, 0, None) \
+        == la.LA_ERR_INVALID_ARG
+    assert la.la_device_status() == la.LA_OK
+
+
+def test_varlen_small_with_empty_sequences():
+    H, d = 3, 128
+    lens = [70, 0, 64, 1, 200, 5]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    q, k, v = inputs.random_qkv(9, 1, H, int(cu[-1]), d, d, dtype=torch.bfloat16)
+    S0 = torch.from_numpy(np.random.default_rng(0).standard_normal((len(lens), H, d, d)).astype(np.float32)) * 0.05
+    O_ref, S_ref = ora.recurrent(q, k, v, S0, cu_seqlens=cu.numpy())
+    for chunk in (64, 128):
+        o, S = gpu_prefill(q, k, v, S0=S0, cu=cu, chunk=chunk, max_seqlen=max(lens))
+        assert nerr(o, O_ref) <= BF16_TOL
+        assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
+        assert torch.equal(S.reshape(S_ref.shape)[1].cpu(), S0[1])  # empty sequence untouched
+
+
+def test_prefill_then_decode_equals_longer_prefill():
+    B, H, T, n, d = 2, 4, 150, 12, 128
+    q, k, v = inputs.random_qkv(17, B, H, T + n, d, d, dtype=torch.bfloat16)
+    o_long, S_long = gpu_prefill(q, k, v, chunk=64)
+    _, S = gpu_prefill(q[:, :, :T], k[:, :, :T], v[:, :, :T], chunk=64)
+    S = S.reshape(B, H, d, d)
+    for t in range(T, T + n):
+        od = torch.empty(B, H, d, dtype=torch.bfloat16, device="cuda")
+        la.la_decode_step(q[:, :, t].cuda().contiguous(), k[:, :, t].cuda().contiguous(),
+                          v[:, :, t].cuda().contiguous(), od, S)
+        assert nerr(od, o_long[:, :, t].float().cpu().numpy()) <= BF16_TOL
+    assert nerr(S, S_long.reshape(B, H, d, d).cpu().numpy()) <= BF16_TOL
+    O_ref, S_ref = ora.recurrent(q, k, v)
+    assert nerr(S, S_ref) <= BF16_TOL
+
+
+# ------------------------------------------- the five workloads ----
+
+def _decode_run(wl, S_dev, units, steps, sample):
+    """Run `steps` decode steps on all `units` states; oracle on `sample` units."""
+    Sd = S_dev.reshape(units, wl.d, wl.d)
+    Sr = {u: Sd[u].double().cpu().numpy() for u in sample}
+    worst = 0.0
+    for step in range(steps):
+        q, k, v = inputs.decode_token(wl, step, units=units)
+        od = torch.empty(units, 1, wl.d, dtype=wl.torch_dtype, device="cuda")
+        la.la_decode_step(q.cuda()[:, None], k.cuda()[:, None], v.cuda()[:, None], od, Sd)
+        oc = od.float().cpu()
+        for u in sample:
+            o_ref, Sr[u] = ora.decode_step(q[u], k[u], v[u], Sr[u])
+            worst = max(worst, nerr(oc[u, 0], o_ref))
+    Sc = Sd.cpu()
+    worst_s = max(nerr(Sc[u], Sr[u]) for u in sample)
+    return worst, worst_s
+
+
+def test_workload_b4h8_t2048_d64_full():
+    wl = WL["b4h8_t2048_d64"]
+    q, k, v, _ = inputs.prefill_inputs(wl)
+    assert la.la_prefill_path(wl.torch_dtype, wl.d, wl.d, wl.chunk) == "tc"
+    O_ref, S_ref = ora.recurrent(q, k, v)
+    o, S = gpu_prefill(q, k, v, chunk=wl.chunk)
+    assert nerr(o, O_ref) <= BF16_TOL
+    assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
+    e_o, e_s = _decode_run(wl, S, inputs.decode_units(wl), wl.decode_steps, sample=[0, 13, 31])
+    assert e_o <= BF16_TOL and e_s <= BF16_TOL
+
+
+@pytest.mark.parametrize("chunk", [64, 128])
+def test_workload_b8h16_t8192_d128_sampled(chunk):
+    wl = WL["b8h16_t8192_d128_knorm"]
+    q, k, v, _ = inputs.prefill_inputs(wl)
+    o, S = gpu_prefill(q, k, v, chunk=chunk)
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    sample = [0, 37, 64, 127]
+    for u, (O_ref, S_ref) in zip(sample, oracle_units(wl, sample)):
+        b, h = divmod(u, wl.H)
+        assert nerr(o[b, h], O_ref) <= BF16_TOL, u
+        assert nerr(S[u], S_ref) <= BF16_TOL, u
+    if chunk == 64:
+        e_o, e_s = _decode_run(wl, S, inputs.decode_units(wl), 32, sample=[0, 77])
+        assert e_o <= BF16_TOL and e_s <= BF16_TOL
+
+
+def test_workload_b1h32_t131072_d128_sampled():
+    wl = WL["b1h32_t131072_d128"]
+    q, k, v, _ = inputs.prefill_inputs(wl)
+    o, S = gpu_prefill(q, k, v, chunk=wl.chunk)
+    assert torch.isfinite(S).all()
+    sample = [0, 31]
+    for u, (O_ref, S_ref) in zip(sample, oracle_units(wl, sample)):
+        assert nerr(o[0, u], O_ref) <= BF16_TOL, u
+        assert nerr(S[u], S_ref) <= BF16_TOL, u
+
+
+def test_workload_varlen64_h32_d128_sampled():
+    wl = WL["varlen64_h32_d128"]
+    q, k, v, cu = inputs.prefill_inputs(wl)
+    lens = (cu[1:] - cu[:-1]).numpy()
+    o, S = gpu_prefill(q, k, v, cu=cu, chunk=wl.chunk, max_seqlen=int(lens.max()))
+    assert torch.isfinite(S).all()
+    sample = [0, 5 * wl.H + 7, int(np.argmax(lens)) * wl.H + 31, int(np.argmin(lens)) * wl.H + 2]
+    for u, (O_ref, S_ref) in zip(sample, oracle_units(wl, sample)):
+        h, r0, L = inputs.unit_rows(wl, u)
+        assert nerr(o[0, h, r0:r0 + L], O_ref) <= BF16_TOL, u
+        assert nerr(S.reshape(-1, wl.d, wl.d)[u], S_ref) <= BF16_TOL, u
+    # decode: the 64 x 32 prefilled states, repeated 4 times -> 256 x 32 units
+    units = inputs.decode_units(wl)
+    Sdec = S.reshape(-1, wl.d, wl.d).repeat(wl.decode_repeat, 1, 1).contiguous()
+    e_o, e_s = _decode_run(wl, Sdec, units, 16, sample=[0, units - 1])
+    assert e_o <= BF16_TOL and e_s <= BF16_TOL

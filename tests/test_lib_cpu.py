@@ -1,0 +1,77 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point declared in include/linattn.h, and answers host-only
+queries (status strings, kernel choice, argument validation before launch)."""
+import os
+import re
+
+import pytest
+import torch
+
+import recurrent_decode_la_b200 as la
+from recurrent_decode_la_b200 import build as labuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "linattn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(la_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    labuild.build()
+    return la.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    syms = _declared_symbols()
+    assert "la_prefill" in syms and "la_decode_step" in syms and "la_state_init" in syms
+    for name in syms:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert la.la_status_string(code)
+    assert la.la_status_string(la.LA_ERR_TIMEOUT) == "device wait timed out"
+
+
+def test_kernel_choice():
+    assert la.la_prefill_path(torch.bfloat16, 128, 128, 64) == "tc"
+    assert la.la_prefill_path(torch.bfloat16, 64, 64, 128) == "tc"
+    assert la.la_prefill_path(torch.bfloat16, 128, 128, 128) == "tc"
+    assert la.la_prefill_path(torch.bfloat16, 96, 96, 64) == "simt"
+    assert la.la_prefill_path(torch.float32, 128, 128, 64) == "simt"
+    assert la.la_prefill_path(torch.float32, 2, 2, 4) == "simt"
+    assert la.la_prefill_path(torch.bfloat16, 256, 256, 64) == "unsupported"
+    assert la.la_prefill_path(torch.float32, 128, 128, 256) == "unsupported"   # tiles exceed smem
+    assert la.la_resolve_chunk(torch.bfloat16, 128, 128, 0) == 64
+    assert la.la_resolve_chunk(torch.bfloat16, 128, 128, 96) == 96
+
+
+def test_argument_checks_before_any_launch(lib):
+    # all of these are rejected on the host: no device is touched
+    assert lib.la_prefill(None, None, None, None, None, 1, 1, 1, 8, 64, 64, None, 0, 0, 64, None, 0, None) \
+        == la.LA_ERR_INVALID_ARG
+    assert lib.la_prefill(None, None, None, None, None, 9, 1, 1, 8, 64, 64, None, 0, 0, 64, None, 0, None) \
+        == la.LA_ERR_INVALID_ARG
+    assert lib.la_prefill(None, None, None, None, None, 1, -1, 1, 8, 64, 64, None, 0, 0, 64, None, 0, None) \
+        == la.LA_ERR_INVALID_ARG
+    assert lib.la_prefill(None, None, None, None, None, 1, 2, 1, 8, 64, 64, 16, 1, 8, 64, None, 0, None) \
+        == la.LA_ERR_INVALID_ARG  # cu_seqlens needs B == 1
+    assert lib.la_decode_step(None, None, None, None, None, 1, 1, 1, 64, 64, None) == la.LA_ERR_INVALID_ARG
+    assert lib.la_decode_step(None, None, None, None, None, 1, 1, 1, 256, 64, None) == la.LA_ERR_UNSUPPORTED
+    assert lib.la_state_init(None, None, 4, 8, 8, None) == la.LA_ERR_INVALID_ARG
+    # empty work is a successful no-op, even with NULL pointers
+    assert lib.la_prefill(None, None, None, None, None, 1, 0, 4, 8, 64, 64, None, 0, 0, 64, None, 0, None) == la.LA_OK
+    assert lib.la_prefill(None, None, None, None, None, 1, 1, 4, 0, 64, 64, None, 0, 0, 64, None, 0, None) == la.LA_OK
+    assert lib.la_state_init(None, None, 0, 8, 8, None) == la.LA_OK
+    assert lib.la_prefill_workspace_size(1, 8, 16, 8192, 128, 128, 0, 64) == 0
+
+
+def test_binding_rejects_cpu_tensors():
+    x = torch.zeros(1, 1, 4, 8)
+    with pytest.raises(ValueError):
+        la.la_prefill(x, x, x, x.clone(), torch.zeros(1, 8, 8))
