@@ -23,7 +23,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -41,11 +40,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--chunk", type=int, default=0, help="0 = the workload's chunk size")
+    ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
+    ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end run")
     ap.add_argument("--decode-steps", type=int, default=-1, help="-1 = the workload's count")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -68,63 +69,66 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons of one GPU
+    every 100 ms through NVML (read-only queries) while the timed region runs."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
-        self.t = None
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._t = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nv = nv
+            u = self.uuid if self.uuid is None or self.uuid.startswith("GPU-") else "GPU-" + self.uuid
+            self._h = nv.nvmlDeviceGetHandleByUUID(u) if u else nv.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception as e:  # no NVML: report no samples
+            self.error = repr(e)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((mhz, mask))
+            except Exception as e:
+                self.error = repr(e)
+            self._stop.wait(0.1)
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            if self.t is not None:
-                self.t.join(timeout=2)
+        self._stop.set()
+        if self._t is not None:
+            self._t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, p in zip(names, parts[5:9]):
-                if p.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "error": self.error}
+        nv = self._nv
+        reasons = set()
+        for _, mask in self.samples:
+            for name, const in self.REASONS.items():
+                if hasattr(nv, const) and mask & getattr(nv, const):
+                    reasons.add(name)
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "sm_min_mhz": min(mhz),
+                "reasons": sorted(reasons), "samples": len(mhz)}
 
 
 def dist_env():
@@ -309,7 +313,8 @@ def run_ours(args, wl, world, rank, local):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(getattr(torch.cuda.get_device_properties(dev), "uuid", None) and
+                      str(torch.cuda.get_device_properties(dev).uuid)) as clk:
         with torch.cuda.stream(stream):
             t_start.record(stream)
             for i in range(args.steps):
@@ -463,13 +468,14 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
         od_h.copy_(od, non_blocking=True)
         st_h.copy_(st, non_blocking=True)
 
+    n_steps = max(1, min(args.steps, args.e2e_steps))
     with torch.cuda.stream(stream):
-        for _ in range(max(1, args.warmup)):
+        for _ in range(3):
             step()
         stream.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(n_steps):
             step()
         e1.record(stream)
     stream.synchronize()
@@ -477,14 +483,18 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
     h2d = sum(x.numel() * x.element_size() for x in pins)
     d2h = o_h.numel() * o_h.element_size() + od_h.numel() * od_h.element_size() + st_h.numel() * 4
     tokens = B * T + B * dsteps
-    return {"value": world * args.steps * tokens / (ms * 1e-3), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps}
+    return {"value": world * n_steps * tokens / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / n_steps,
+            "steps": n_steps}
 
 
 def main(argv=None):
     args = parse_args(argv)
     from recurrent_decode_la_b200 import inputs
     wl = inputs.WORKLOADS[args.workload]
+    if args.batch > 0:
+        import dataclasses
+        wl = dataclasses.replace(wl, name=f"{wl.name}_b{args.batch}", B=args.batch)
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
