@@ -44,7 +44,9 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--chunk", type=int, default=0, help="0 = the workload's chunk size")
+    ap.add_argument("--chunk", type=int, default=0, help="0 = the library's default for the shape")
+    ap.add_argument("--sweep-chunks", default="64,128",
+                    help="also time the prefill alone at these chunk sizes ('' = none)")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
     ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end run")
     ap.add_argument("--decode-steps", type=int, default=-1, help="-1 = the workload's count")
@@ -255,7 +257,7 @@ def run_ours(args, wl, world, rank, local):
                                 device_id=dev)
     peaks, peak_src = load_peaks()
     B, H, T, d = wl.B, wl.H, wl.T, wl.d
-    chunk = args.chunk or wl.chunk
+    chunk = args.chunk or la.la_resolve_chunk(wl.torch_dtype, wl.d, wl.d, 0)
     dsteps = wl.decode_steps if args.decode_steps < 0 else args.decode_steps
     units = B * H
     elem = 2 if wl.dtype == "bf16" else 4
@@ -296,16 +298,19 @@ def run_ours(args, wl, world, rank, local):
     if la.la_device_status(stream) != la.LA_OK:
         raise RuntimeError("device status not ok after warm-up")
 
-    g_pre, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    g_pre = torch.cuda.CUDAGraph()
+    g_dec = torch.cuda.CUDAGraph() if dsteps else None
     with torch.cuda.graph(g_pre, stream=stream):
         prefill_phase(torch.cuda.current_stream())
-    with torch.cuda.graph(g_dec, stream=stream):
-        decode_phase(torch.cuda.current_stream())
+    if g_dec is not None:
+        with torch.cuda.graph(g_dec, stream=stream):
+            decode_phase(torch.cuda.current_stream())
 
     for _ in range(args.warmup):
         with torch.cuda.stream(stream):
             g_pre.replay()
-            g_dec.replay()
+            if g_dec is not None:
+                g_dec.replay()
     stream.synchronize()
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -321,7 +326,8 @@ def run_ours(args, wl, world, rank, local):
                 ev[i][0].record(stream)
                 g_pre.replay()
                 ev[i][1].record(stream)
-                g_dec.replay()
+                if g_dec is not None:
+                    g_dec.replay()
                 ev[i][2].record(stream)
             t_end.record(stream)
         torch.cuda.synchronize()
@@ -384,6 +390,10 @@ def run_ours(args, wl, world, rank, local):
     result["roofline_prefill"] = roof_pre
     result["clocks"] = clk.summary()
 
+    if args.sweep_chunks:
+        result["chunk_sweep"] = chunk_sweep(la, torch, stream, q, k, v, o, state, wl,
+                                            [int(c) for c in args.sweep_chunks.split(",")], peaks)
+
     if not args.no_cold_decode and dsteps:
         result["decode_cold"] = cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_src)
 
@@ -400,6 +410,34 @@ def run_ours(args, wl, world, rank, local):
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def chunk_sweep(la, torch, stream, q, k, v, o, state, wl, chunks, peaks):
+    """Prefill alone at several chunk sizes (C never changes the result, only
+    the cost): CUDA-event time of one launch, median of 20 after 3 warm-ups."""
+    out = {}
+    units, d = wl.B * wl.H, wl.d
+    elem = 2 if wl.dtype == "bf16" else 4
+    byts = prefill_bytes(units, wl.T, d, d, elem)
+    for c in chunks:
+        path = la.la_prefill_path(wl.torch_dtype, d, d, c, q, k, v, o)
+        ts = []
+        with torch.cuda.stream(stream):
+            for i in range(23):
+                la.la_state_init(state, None, stream=stream)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                la.la_prefill(q, k, v, o, state, chunk=c, stream=stream)
+                e1.record(stream)
+                e1.synchronize()
+                if i >= 3:
+                    ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        flops = prefill_flops_dense(units, wl.T, d, d, c)
+        out[str(c)] = {"kernel": path, "ms": ms, "tokens_per_s": wl.B * wl.T / (ms * 1e-3),
+                       "hbm_frac": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                       "tensor_frac_burst_dense": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+    return out
 
 
 def cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_src):

@@ -82,11 +82,22 @@ int default_chunk(la_dtype dtype, int dk, int dv) {
         const int c = atoi(e);
         if (c > 0) return c;
     }
-    if (dtype == LA_BF16 && dk == dv && (dk == 64 || dk == 128)) return 64;
+    // bf16 tensor-core path: 128-token chunks run full-rate M = 128 MMAs with
+    // P kept in tensor memory (the measured fastest chunk on B200).
+    if (dtype == LA_BF16 && dk == dv && (dk == 64 || dk == 128)) return 128;
     return dk <= 32 && dv <= 32 ? 32 : 16;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Event-trace buffer of the tensor-core prefill; set only through the
+// debugging hook of LINATTN_TRACE builds.
+struct TraceBuf {
+    unsigned long long* buf = nullptr;
+    unsigned int* count = nullptr;
+    unsigned int cap = 0;
+};
+TraceBuf g_trace;
 
 enum Path { kTc, kSimt, kUnsupported };
 
@@ -183,6 +194,9 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     p.cu = cu_seqlens;
     p.chunk = c;
     p.timeout_ns = wait_timeout_ns();
+    p.trace = g_trace.buf;
+    p.trace_count = g_trace.count;
+    p.trace_cap = g_trace.cap;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int sms = current_sm_count();
     cudaError_t e;
@@ -212,6 +226,18 @@ la_status la_decode_step(const void* q, const void* k, const void* v, void* o, f
                                   current_sm_count(), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? LA_OK : cuda_fail(e);
 }
+
+#ifdef LINATTN_TRACE
+// Debugging hook of trace builds only (not part of the ABI): record events of
+// CTA 0 of later tensor-core prefill launches into `buf` (`cap` records) and
+// count them in `*count` (device memory, zeroed by the caller).
+la_status la_debug_set_trace(unsigned long long* buf, unsigned int* count, unsigned int cap) {
+    g_trace.buf = buf;
+    g_trace.count = count;
+    g_trace.cap = cap;
+    return LA_OK;
+}
+#endif
 
 la_status la_device_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

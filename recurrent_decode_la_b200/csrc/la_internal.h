@@ -26,6 +26,10 @@ struct PrefillProblem {
     const int32_t* cu;  // nullptr for dense input
     int chunk;
     uint64_t timeout_ns;
+    // Event trace of CTA 0 (builds with LINATTN_TRACE only; nullptr otherwise).
+    unsigned long long* trace;
+    unsigned int* trace_count;
+    unsigned int trace_cap;
 };
 
 cudaError_t launch_prefill_simt(const PrefillProblem& p, int num_sms, cudaStream_t s);

@@ -12,12 +12,14 @@
 // the state is copied out once as a bf16 operand for the next chunk's Q S.
 //
 // One persistent CTA per SM walks units (one sequence of one head) with a
-// static stride.  Warp roles (384 threads):
-//   warp 0      TMA producer: Q/K/V chunk tiles into an NS-deep ring
-//   warp 1      MMA issuer (one thread) and TMEM owner
-//   warps 4-7   "state" warpgroup: causal mask -> P, state hop S -> bf16,
-//               S_0 in and S_T out
-//   warps 8-11  "output" warpgroup: O TMEM -> bf16 -> smem -> TMA store
+// static stride.  Warp roles (512 threads):
+//   warp 0       TMA producer: Q/K/V chunk tiles into an NS-deep ring
+//   warp 1       MMA issuer (one thread) and TMEM owner
+//   warps 4-7    "mask" warpgroup: scores -> causal mask -> bf16 P
+//   warps 8-11   "state" warpgroup: S_0 in, state hop S -> bf16 operand, S_T out
+//   warps 12-15  "output" warpgroup: O TMEM -> bf16 -> smem -> TMA store
+// The mask and the state hop run in different warpgroups so that the two
+// per-chunk chains (scores -> P -> P V, and S -> bf16 S -> next Q S) overlap.
 // Every wait is an mbarrier wait bounded by a timeout; on expiry the kernel
 // records the error word, every role winds down, outstanding copies and
 // MMAs are drained (bounded), TMEM is freed and the kernel returns.
@@ -26,17 +28,38 @@
 
 namespace la {
 
+// Optional event trace (compiled in only with -DLINATTN_TRACE): CTA 0 stores
+// the SM clock of event `ev` of chunk `g` at trace[ev * (cap / 64) + g]
+// (plain stores: no atomics on the traced threads).
+#ifdef LINATTN_TRACE
+#define LA_TRACE(ev, g)                                                                         \
+    do {                                                                                        \
+        if (p.trace && blockIdx.x == 0 && (g) < static_cast<int64_t>(p.trace_cap / 64))          \
+            p.trace[(ev) * (p.trace_cap / 64) + (g)] = clock64();                               \
+    } while (0)
+#else
+#define LA_TRACE(ev, g) \
+    do {                \
+    } while (0)
+#endif
+
 template <int C, int D>
 struct TcCfg {
-    static constexpr int kThreads = 384;
+    static constexpr int kThreads = 512;
     static constexpr int PANEL = C * 128;  // one 64-column panel of a chunk tile (bytes)
     static constexpr int NPAN = D / 64;
     static constexpr int TILE = C * D * 2;
     static constexpr int STAGE = 3 * TILE;  // Q, K, V of one chunk
-    static constexpr int NS = (C == 64 && D == 64) ? 6 : (C == 64 ? 3 : (D == 64 ? 2 : 1));
-    static constexpr int PB = 2;                           // P buffers
+    // C = 128: P stays in tensor memory (written over the fp32 scores it came
+    // from, read by the P V MMA straight from TMEM) and O is staged for its
+    // TMA store in the chunk's own Q tile, which is dead by then; the shared
+    // memory this frees buys a deeper Q/K/V ring.  C = 64 (M = 64 tiles) keeps
+    // P and the O staging in their own shared-memory buffers.
+    static constexpr bool PT = (C == 128);
+    static constexpr int NS = PT ? (D == 128 ? 2 : 4) : (D == 64 ? 6 : 3);
+    static constexpr int PB = PT ? 0 : 2;                       // P buffers in smem
     static constexpr int OB = (C == 128 && D == 128) ? 1 : 2;  // O accumulators in TMEM
-    static constexpr int OSB = (C == 128 && D == 128) ? 1 : 2;  // O staging buffers
+    static constexpr int OSB = PT ? 0 : 2;                      // O staging buffers in smem
     static constexpr int P_BYTES = C * C * 2;
     static constexpr int P_PANEL = C * 128;
     static constexpr int SB_BYTES = D * D * 2;
@@ -47,7 +70,7 @@ struct TcCfg {
     static constexpr int OFF_SB = OFF_P + PB * P_BYTES;
     static constexpr int OFF_OST = OFF_SB + SB_BYTES;
     static constexpr int OFF_BAR = OFF_OST + OSB * OST_BYTES;
-    static constexpr int NBAR = 40;
+    static constexpr int NBAR = 48;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
     // tensor memory columns (fp32, 128 lanes)
@@ -73,7 +96,8 @@ struct TcCfg {
     static constexpr int B_OEMPTY = 30;    // [2] O read out
     static constexpr int B_OSTFULL = 32;   // [2] O staging written
     static constexpr int B_OSTFREE = 34;   // [2] O staging read by the TMA store
-    static constexpr int B_MMADONE = 36;   // drain at teardown
+    static constexpr int B_MMADONE = 36;   // [2] drain at teardown (one per issuing thread)
+    static constexpr int B_ZERO = 40;      // [NS] rows past the sequence end zeroed in K, V
 };
 
 struct Unit {
@@ -105,7 +129,7 @@ __device__ __forceinline__ int acc_row(int sub, int lane) {
 }
 
 template <int C, int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV,
@@ -125,7 +149,10 @@ __global__ void __launch_bounds__(384, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::NS; ++s) {
             mbar_init(&bar[Cfg::B_FULL + s], 1);
-            mbar_init(&bar[Cfg::B_EMPTY + s], 1);
+            // released by the state stream's K^T V and by the chunk's last
+            // other reader (the P V MMA, or the O store that reuses Q's tile)
+            mbar_init(&bar[Cfg::B_EMPTY + s], 2);
+            mbar_init(&bar[Cfg::B_ZERO + s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar[Cfg::B_AFULL + b], 1);
@@ -142,6 +169,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(&bar[Cfg::B_SBFULL], 4);
         mbar_init(&bar[Cfg::B_SBEMPTY], 1);
         mbar_init(&bar[Cfg::B_MMADONE], 1);
+        mbar_init(&bar[Cfg::B_MMADONE + 1], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -199,6 +227,7 @@ __global__ void __launch_bounds__(384, 1)
                                     &tmV, &bar[Cfg::B_FULL + s], pn * 64, row, un.group);
                     }
                     last_g[s] = g;
+                    LA_TRACE(1, g);
                 }
             }
             if (!ok || *abort_flag) {
@@ -208,129 +237,324 @@ __global__ void __launch_bounds__(384, 1)
                         mbar_wait_drain(&bar[Cfg::B_FULL + s], (last_g[s] / Cfg::NS) & 1, tmo);
             }
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
+    } else if (warp == 1 || warp == 2) {
+        // ----------------------------------------------------- MMA issuers
+        // Two threads issue tcgen05 MMAs; an issuing thread blocks while the
+        // tensor pipe is busy, so splitting the work keeps one stream going
+        // while the other waits on a warpgroup:
+        //   warp 1 (chunk attention): A = Q K^T, O = Q S_prev, O += P V.  The
+        //     scores of chunk g+1 are issued between the two O MMAs of chunk g
+        //     when its tiles have already landed (never blocking on a load).
+        //   warp 2 (state carry): rows past a sequence end are zeroed in K and
+        //     V, then S += K^T V as soon as the previous state has been read.
         constexpr uint32_t kIdQK = idesc_bf16_f32(C, C, false, false);
         constexpr uint32_t kIdKV = idesc_bf16_f32(D, D, true, true);
         constexpr uint32_t kIdQS = idesc_bf16_f32(C, D, false, true);
         constexpr uint32_t kIdPV = idesc_bf16_f32(C, D, false, true);
-        const uint32_t tm_S = tmem + Cfg::TM_S;
-        int64_t g = 0;
+        constexpr bool kLookahead = Cfg::NS >= 2;
+        const bool attn = (warp == 1);
         bool ok = true;
         bool issued_any = false;
-        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
-            const Unit un = get_unit(p, u);
-            const int nch = (un.len + C - 1) / C;
-            for (int c = 0; c < nch; ++c, ++g) {
+        // (unit, chunk) walk
+        struct Cursor {
+            int64_t u;
+            int c, nch, nv;
+            int64_t g;
+            bool valid;
+        };
+        auto first = [&](Cursor& k) {
+            k.g = 0;
+            k.c = 0;
+            for (k.u = blockIdx.x; k.u < p.n_units; k.u += gridDim.x) {
+                const Unit un = get_unit(p, k.u);
+                k.nch = (un.len + C - 1) / C;
+                if (k.nch > 0) {
+                    k.nv = min(C, un.len);
+                    k.valid = true;
+                    return;
+                }
+            }
+            k.valid = false;
+        };
+        auto advance = [&](Cursor& k) {
+            ++k.g;
+            if (++k.c < k.nch) {
+                const Unit un = get_unit(p, k.u);
+                k.nv = min(C, un.len - k.c * C);
+                return;
+            }
+            k.c = 0;
+            for (k.u += gridDim.x; k.u < p.n_units; k.u += gridDim.x) {
+                const Unit un = get_unit(p, k.u);
+                k.nch = (un.len + C - 1) / C;
+                if (k.nch > 0) {
+                    k.nv = min(C, un.len);
+                    return;
+                }
+            }
+            k.valid = false;
+        };
+
+        if (!attn) {
+            // ------------------------------------------------ state stream
+            const uint32_t tm_S = tmem + Cfg::TM_S;
+            Cursor k;
+            for (first(k); ok && k.valid; advance(k)) {
+                const int64_t g = k.g;
                 const int s = static_cast<int>(g % Cfg::NS);
-                const int nv = min(C, un.len - c * C);
-                if (!mbar_wait_warp(&bar[Cfg::B_FULL + s], (g / Cfg::NS) & 1, abort_flag, tmo,
-                                    0x200 + s)) {
+                if (!mbar_wait_warp(&bar[Cfg::B_FULL + s], (g / Cfg::NS) & 1, abort_flag, tmo, 0x200 + s)) {
                     ok = false;
                     break;
                 }
-                if (nv < C) {
+                if (k.nv < C) {
                     // Rows past the end of the sequence must not reach the
-                    // state: zero them in the K and V tiles.
-                    const int nrow = C - nv;
+                    // state (nor, through P = 0 on them, the output).
+                    const int nrow = C - k.nv;
                     const int per_tile = nrow * Cfg::NPAN * 8;  // 16-byte pieces
                     for (int i = lane; i < 2 * per_tile; i += 32) {
                         const int t = i / per_tile;
                         const int r = i % per_tile;
-                        const int row = nv + r / (Cfg::NPAN * 8);
+                        const int row = k.nv + r / (Cfg::NPAN * 8);
                         const int pn = (r / 8) % Cfg::NPAN;
                         const int ch = r % 8;
                         const uint32_t base = t == 0 ? stage_k(s) : stage_v(s);
                         st_shared_v4(base + pn * Cfg::PANEL + row * 128 + ch * 16, 0u, 0u, 0u, 0u);
                     }
                     fence_proxy_async_smem();
-                    __syncwarp();
                 }
+                __syncwarp();
+                int okw = 1;
                 if (lane == 0) {
-                    const int b = static_cast<int>(g & 1);
-                    const int ob = static_cast<int>(g % Cfg::OB);
-                    const uint32_t qb = stage_q(s), kb = stage_k(s), vb = stage_v(s);
-                    // (1) A = Q K^T
-                    if (g >= 2 && !mbar_wait(&bar[Cfg::B_AEMPTY + b], ((g >> 1) + 1) & 1,
-                                             abort_flag, tmo, 0x210 + b)) {
-                        ok = false;
+                    mbar_arrive(&bar[Cfg::B_ZERO + s]);
+                    if (!mbar_wait(&bar[Cfg::B_SREAD], g & 1, abort_flag, tmo, 0x220)) okw = 0;
+                    LA_TRACE(4, g);
+                    if (okw) {
+                        tc_fence_after();
+                        const uint32_t kb = stage_k(s), vb = stage_v(s);
+#pragma unroll
+                        for (int ks = 0; ks < C / 16; ++ks)
+                            mma_bf16_ss(tm_S, sdesc_sw128(kb + ks * 2048, Cfg::PANEL, 1024),
+                                        sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024), kIdKV, 1);
+                        mma_commit(&bar[Cfg::B_SFULL]);
+                        mma_commit(&bar[Cfg::B_EMPTY + s]);
+                        issued_any = true;
                     }
-                    if (ok) {
+                }
+                ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
+            }
+        } else {
+            // -------------------------------------------- attention stream
+            auto issue_scores = [&](const Cursor& k) -> bool {
+                const int s = static_cast<int>(k.g % Cfg::NS);
+                if (!mbar_wait_warp(&bar[Cfg::B_FULL + s], (k.g / Cfg::NS) & 1, abort_flag, tmo, 0x208 + s))
+                    return false;
+                if (lane == 0) LA_TRACE(2, k.g);
+                int okw = 1;
+                if (lane == 0) {
+                    const int b = static_cast<int>(k.g & 1);
+                    if (k.g >= 2 && !mbar_wait(&bar[Cfg::B_AEMPTY + b], ((k.g >> 1) + 1) & 1, abort_flag, tmo,
+                                               0x210 + b))
+                        okw = 0;
+                    if (okw) {
                         tc_fence_after();
                         const uint32_t tm_A = tmem + Cfg::TM_A + b * C;
+                        const uint32_t qb = stage_q(s), kb = stage_k(s);
 #pragma unroll
                         for (int ks = 0; ks < D / 16; ++ks) {
                             const uint32_t off = (ks >> 2) * Cfg::PANEL + (ks & 3) * 32;
-                            mma_bf16_ss(tm_A, sdesc_sw128(qb + off, 16, 1024),
-                                        sdesc_sw128(kb + off, 16, 1024), kIdQK, ks > 0);
+                            mma_bf16_ss(tm_A, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                                        kIdQK, ks > 0);
                         }
                         mma_commit(&bar[Cfg::B_AFULL + b]);
-                        issued_any = true;
+                        LA_TRACE(3, k.g);
                     }
-                    // (2) S += K^T V
-                    if (ok && !mbar_wait(&bar[Cfg::B_SREAD], g & 1, abort_flag, tmo, 0x220))
-                        ok = false;
-                    if (ok) {
+                }
+                return __shfl_sync(0xffffffffu, okw, 0) != 0;
+            };
+
+            Cursor cur, nxt;
+            first(cur);
+            nxt = cur;
+            if (cur.valid) {
+                ok = issue_scores(cur);
+                issued_any = true;
+                advance(nxt);
+            }
+            while (ok && cur.valid) {
+                const int64_t g = cur.g;
+                const int s = static_cast<int>(g % Cfg::NS);
+                const int b = static_cast<int>(g & 1);
+                const int ob = static_cast<int>(g % Cfg::OB);
+                const uint32_t tm_O = tmem + Cfg::TM_O + ob * D;
+                bool next_scored = false;
+                int okw = 1;
+                if (lane == 0) {
+                    // O = Q S_prev
+                    if (g >= Cfg::OB &&
+                        !mbar_wait(&bar[Cfg::B_OEMPTY + ob], ((g / Cfg::OB) + 1) & 1, abort_flag, tmo, 0x230 + ob))
+                        okw = 0;
+                    if (okw && !mbar_wait(&bar[Cfg::B_SBFULL], g & 1, abort_flag, tmo, 0x240)) okw = 0;
+                    LA_TRACE(5, g);
+                    if (okw) {
                         tc_fence_after();
-#pragma unroll
-                        for (int ks = 0; ks < C / 16; ++ks) {
-                            mma_bf16_ss(tm_S, sdesc_sw128(kb + ks * 2048, Cfg::PANEL, 1024),
-                                        sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024), kIdKV, 1);
-                        }
-                        mma_commit(&bar[Cfg::B_SFULL]);
-                    }
-                    // (3) O = Q S_prev
-                    if (ok && g >= Cfg::OB &&
-                        !mbar_wait(&bar[Cfg::B_OEMPTY + ob], ((g / Cfg::OB) + 1) & 1, abort_flag,
-                                   tmo, 0x230 + ob))
-                        ok = false;
-                    if (ok && !mbar_wait(&bar[Cfg::B_SBFULL], g & 1, abort_flag, tmo, 0x240))
-                        ok = false;
-                    const uint32_t tm_O = tmem + Cfg::TM_O + ob * D;
-                    if (ok) {
-                        tc_fence_after();
+                        const uint32_t qb = stage_q(s);
 #pragma unroll
                         for (int ks = 0; ks < D / 16; ++ks) {
                             const uint32_t off = (ks >> 2) * Cfg::PANEL + (ks & 3) * 32;
                             mma_bf16_ss(tm_O, sdesc_sw128(qb + off, 16, 1024),
-                                        sdesc_sw128(sb_base + ks * 2048, Cfg::SB_PANEL, 1024),
-                                        kIdQS, ks > 0);
+                                        sdesc_sw128(sb_base + ks * 2048, Cfg::SB_PANEL, 1024), kIdQS, ks > 0);
                         }
                         mma_commit(&bar[Cfg::B_SBEMPTY]);
                     }
-                    // (4) O += P V
-                    if (ok && !mbar_wait(&bar[Cfg::B_PFULL + b], (g >> 1) & 1, abort_flag, tmo,
-                                         0x250 + b))
-                        ok = false;
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t pb = p_base + b * Cfg::P_BYTES;
-#pragma unroll
-                        for (int ks = 0; ks < C / 16; ++ks) {
-                            const uint32_t off = (ks >> 2) * Cfg::P_PANEL + (ks & 3) * 32;
-                            mma_bf16_ss(tm_O, sdesc_sw128(pb + off, 16, 1024),
-                                        sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024), kIdPV, 1);
-                        }
-                        mma_commit(&bar[Cfg::B_PEMPTY + b]);
-                        mma_commit(&bar[Cfg::B_OFULL + ob]);
-                        mma_commit(&bar[Cfg::B_EMPTY + s]);
+                }
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) break;
+                // Look ahead without blocking: if the next chunk's tiles have
+                // landed, issue its scores now so the mask warpgroup can start
+                // on them while this chunk's P V runs.
+                if (kLookahead && nxt.valid) {
+                    int ready = 0;
+                    if (lane == 0)
+                        ready = mbar_try_wait(&bar[Cfg::B_FULL + static_cast<int>(nxt.g % Cfg::NS)],
+                                              (nxt.g / Cfg::NS) & 1) ? 1 : 0;
+                    if (__shfl_sync(0xffffffffu, ready, 0)) {
+                        if (!issue_scores(nxt)) break;
+                        next_scored = true;
                     }
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (lane == 0) {
+                    // O += P V (a partial chunk also waits for its zeroed V rows)
+                    if (!mbar_wait(&bar[Cfg::B_PFULL + b], (g >> 1) & 1, abort_flag, tmo, 0x250 + b)) okw = 0;
+                    if (okw && cur.nv < C &&
+                        !mbar_wait(&bar[Cfg::B_ZERO + s], (g / Cfg::NS) & 1, abort_flag, tmo, 0x260 + s))
+                        okw = 0;
+                    LA_TRACE(6, g);
+                    if (okw) {
+                        tc_fence_after();
+                        const uint32_t vb = stage_v(s);
+                        if constexpr (Cfg::PT) {
+                            const uint32_t tm_P = tmem + Cfg::TM_A + b * C;  // 8 columns per 16 keys
+#pragma unroll
+                            for (int ks = 0; ks < C / 16; ++ks)
+                                mma_bf16_ts(tm_O, tm_P + ks * 8, sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024),
+                                            kIdPV, 1);
+                            mma_commit(&bar[Cfg::B_OFULL + ob]);
+                        } else {
+                            const uint32_t pb = p_base + b * Cfg::P_BYTES;
+#pragma unroll
+                            for (int ks = 0; ks < C / 16; ++ks) {
+                                const uint32_t off = (ks >> 2) * Cfg::P_PANEL + (ks & 3) * 32;
+                                mma_bf16_ss(tm_O, sdesc_sw128(pb + off, 16, 1024),
+                                            sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024), kIdPV, 1);
+                            }
+                            mma_commit(&bar[Cfg::B_PEMPTY + b]);
+                            mma_commit(&bar[Cfg::B_OFULL + ob]);
+                            mma_commit(&bar[Cfg::B_EMPTY + s]);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
                 if (!ok) break;
+                cur = nxt;
+                if (nxt.valid) {
+                    if (!next_scored) {
+                        if (!issue_scores(cur)) break;
+                    }
+                    advance(nxt);
+                }
             }
         }
         if (lane == 0 && issued_any) {
-            // Drain: every MMA issued above has completed before TMEM is freed.
-            mma_commit(&bar[Cfg::B_MMADONE]);
-            mbar_wait_drain(&bar[Cfg::B_MMADONE], 0, tmo);
+            // Drain: every MMA this thread issued has completed before TMEM is freed.
+            mma_commit(&bar[attn ? Cfg::B_MMADONE : Cfg::B_MMADONE + 1]);
+            mbar_wait_drain(&bar[attn ? Cfg::B_MMADONE : Cfg::B_MMADONE + 1], 0, tmo);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------- state / mask warpgroup
+        // ----------------------------------------------------- mask warpgroup
         const int sub = warp & 3;
         const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
         const int rowA = acc_row<C>(sub, lane);  // score / P row
+        int64_t g = 0;
+        bool ok = true;
+        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            const Unit un = get_unit(p, u);
+            const int nch = (un.len + C - 1) / C;
+            for (int c = 0; c < nch; ++c, ++g) {
+                const int b = static_cast<int>(g & 1);
+                // P = mask(A)
+                if (!mbar_wait_warp(&bar[Cfg::B_AFULL + b], (g >> 1) & 1, abort_flag, tmo, 0x310 + b)) {
+                    ok = false;
+                    break;
+                }
+                if (warp == 4 && lane == 0) LA_TRACE(10, g);
+                tc_fence_after();
+                if (!Cfg::PT && g >= 2 &&
+                    !mbar_wait_warp(&bar[Cfg::B_PEMPTY + b], ((g >> 1) + 1) & 1, abort_flag, tmo, 0x320 + b)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t tm_A = tmem + Cfg::TM_A + b * C + lane_off;
+                const uint32_t pb = p_base + b * Cfg::P_BYTES;
+                if constexpr (Cfg::PT) {
+                    // P (bf16 pairs) over the first C/2 columns of the scores:
+                    // half h reads score columns [64h, 64h+64) and writes P
+                    // columns [32h, 32h+32), all of which it has already read.
+#pragma unroll
+                    for (int h = 0; h < C / 64; ++h) {
+                        uint32_t r0[32], r1[32], w[32];
+                        tmem_ld32(tm_A + h * 64, r0);
+                        tmem_ld32(tm_A + h * 64 + 32, r1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int j = h * 64 + 2 * e;
+                            w[e] = pack_bf16x2(j <= rowA ? __uint_as_float(r0[2 * e]) : 0.f,
+                                               j + 1 <= rowA ? __uint_as_float(r0[2 * e + 1]) : 0.f);
+                            const int j2 = j + 32;
+                            w[16 + e] = pack_bf16x2(j2 <= rowA ? __uint_as_float(r1[2 * e]) : 0.f,
+                                                    j2 + 1 <= rowA ? __uint_as_float(r1[2 * e + 1]) : 0.f);
+                        }
+                        tmem_st32(tm_A + h * 32, w);
+                    }
+                    tmem_wait_st();
+                } else
+#pragma unroll
+                for (int cb = 0; cb < C / 32; ++cb) {
+                    uint32_t r[32];
+                    tmem_ld32(tm_A + cb * 32, r);
+                    tmem_wait_ld();
+                    if (rowA >= 0) {
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = cb * 32 + ch * 8 + 2 * e;
+                                const float a0 = (j <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e]) : 0.f;
+                                const float a1 = (j + 1 <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e + 1]) : 0.f;
+                                w[e] = pack_bf16x2(a0, a1);
+                            }
+                            const int col = cb * 32 + ch * 8;
+                            st_shared_v4(pb + (col >> 6) * Cfg::P_PANEL + sw128_off(rowA, (col & 63) >> 3),
+                                         w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bar[Cfg::B_AEMPTY + b]);
+                    mbar_arrive(&bar[Cfg::B_PFULL + b]);
+                    if (warp == 4) LA_TRACE(11, g);
+                }
+            }
+        }
+    } else if (warp >= 8 && warp < 12) {
+        // ---------------------------------------------------- state warpgroup
+        const int sub = warp & 3;
+        const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
         const int rowS = acc_row<D>(sub, lane);  // state row (key index)
         const uint32_t tm_S = tmem + Cfg::TM_S + lane_off;
         int64_t g = 0;
@@ -389,54 +613,12 @@ __global__ void __launch_bounds__(384, 1)
             // ---- chunk loop
             for (int c = 0; c < nch; ++c, ++g) {
                 const bool last = (c == nch - 1);
-                const int b = static_cast<int>(g & 1);
-                // P = mask(A)
-                if (!mbar_wait_warp(&bar[Cfg::B_AFULL + b], (g >> 1) & 1, abort_flag, tmo, 0x310 + b)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (g >= 2 && !mbar_wait_warp(&bar[Cfg::B_PEMPTY + b], ((g >> 1) + 1) & 1, abort_flag,
-                                              tmo, 0x320 + b)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t tm_A = tmem + Cfg::TM_A + b * C + lane_off;
-                const uint32_t pb = p_base + b * Cfg::P_BYTES;
-#pragma unroll
-                for (int cb = 0; cb < C / 32; ++cb) {
-                    uint32_t r[32];
-                    tmem_ld32(tm_A + cb * 32, r);
-                    tmem_wait_ld();
-                    if (rowA >= 0) {
-#pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = cb * 32 + ch * 8 + 2 * e;
-                                const float a0 = (j <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e]) : 0.f;
-                                const float a1 = (j + 1 <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e + 1]) : 0.f;
-                                w[e] = pack_bf16x2(a0, a1);
-                            }
-                            const int col = cb * 32 + ch * 8;
-                            st_shared_v4(pb + (col >> 6) * Cfg::P_PANEL + sw128_off(rowA, (col & 63) >> 3),
-                                         w[0], w[1], w[2], w[3]);
-                        }
-                    }
-                }
-                tc_fence_before();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&bar[Cfg::B_AEMPTY + b]);
-                    mbar_arrive(&bar[Cfg::B_PFULL + b]);
-                }
                 // state hop: S_c out of TMEM
                 if (!mbar_wait_warp(&bar[Cfg::B_SFULL], g & 1, abort_flag, tmo, 0x330)) {
                     ok = false;
                     break;
                 }
+                if (warp == 8 && lane == 0) LA_TRACE(20, g);
                 tc_fence_after();
                 uint32_t pk[D / 2];
 #pragma unroll
@@ -459,10 +641,12 @@ __global__ void __launch_bounds__(384, 1)
                 if (!last) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bar[Cfg::B_SREAD]);
+                    if (warp == 8 && lane == 0) LA_TRACE(21, g);
                     if (!mbar_wait_warp(&bar[Cfg::B_SBEMPTY], g & 1, abort_flag, tmo, 0x340)) {
                         ok = false;
                         break;
                     }
+                    if (warp == 8 && lane == 0) LA_TRACE(22, g);
                     if (rowS >= 0) {
 #pragma unroll
                         for (int ch = 0; ch < D / 8; ++ch) {
@@ -474,15 +658,16 @@ __global__ void __launch_bounds__(384, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bar[Cfg::B_SBFULL]);
+                    if (warp == 8 && lane == 0) LA_TRACE(23, g);
                 }
             }
         }
-    } else if (warp >= 8) {
-        // ------------------------------------------------- output warpgroup
+    } else if (warp >= 12) {
+        // ---------------------------------------------------- output warpgroup
         const int sub = warp & 3;
         const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
         const int row = acc_row<C>(sub, lane);
-        const bool elected = (warp == 8 && lane == 0);
+        const bool elected = (warp == 12 && lane == 0);
         uint16_t* obase = static_cast<uint16_t*>(p.o);
         int64_t g = 0, f = 0;
         bool ok = true;
@@ -497,62 +682,90 @@ __global__ void __launch_bounds__(384, 1)
                     ok = false;
                     break;
                 }
+                if (warp == 12 && lane == 0) LA_TRACE(30, g);
                 tc_fence_after();
-                uint32_t pk[D / 2];
                 const uint32_t tm_O = tmem + Cfg::TM_O + ob * D + lane_off;
-#pragma unroll
-                for (int cb = 0; cb < D / 32; ++cb) {
-                    uint32_t r[32];
-                    tmem_ld32(tm_O + cb * 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[cb * 16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[Cfg::B_OEMPTY + ob]);
                 const int64_t grow0 = static_cast<int64_t>(un.group) * p.rows_per_group + un.row0 + c * C;
+                const int st_s = static_cast<int>(g % Cfg::NS);  // this chunk's Q/K/V stage
                 if (nv == C) {
-                    const int osb = static_cast<int>(f % Cfg::OSB);
-                    if (f >= Cfg::OSB && !mbar_wait_warp(&bar[Cfg::B_OSTFREE + osb], ((f / Cfg::OSB) + 1) & 1,
-                                                         abort_flag, tmo, 0x410 + osb)) {
+                    // Full chunk: TMEM -> bf16 -> swizzled staging tile -> TMA store.
+                    const int osb = static_cast<int>(f & 1);
+                    if (!Cfg::PT && f >= Cfg::OSB &&
+                        !mbar_wait_warp(&bar[Cfg::B_OSTFREE + osb], ((f / 2) + 1) & 1, abort_flag, tmo,
+                                        0x410 + osb)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t stg = ost_base + osb * Cfg::OST_BYTES;
-                    if (row >= 0) {
+                    // C = 128 stages O in the chunk's own Q tile: its last readers
+                    // (the Q K^T and Q S MMAs) completed before O did.
+                    const uint32_t stg = Cfg::PT ? stage_q(st_s) : ost_base + osb * Cfg::OST_BYTES;
 #pragma unroll
-                        for (int ch = 0; ch < D / 8; ++ch) {
-                            const int col = ch * 8;
-                            st_shared_v4(stg + (col >> 6) * Cfg::PANEL + sw128_off(row, (col & 63) >> 3),
-                                         pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        uint32_t r[32];
+                        tmem_ld32(tm_O + cb * 32, r);
+                        tmem_wait_ld();
+                        if (row >= 0) {
+#pragma unroll
+                            for (int ch = 0; ch < 4; ++ch) {
+                                const int col = cb * 32 + ch * 8;
+                                st_shared_v4(stg + (col >> 6) * Cfg::PANEL + sw128_off(row, (col & 63) >> 3),
+                                             pack_bf16x2(__uint_as_float(r[ch * 8 + 0]), __uint_as_float(r[ch * 8 + 1])),
+                                             pack_bf16x2(__uint_as_float(r[ch * 8 + 2]), __uint_as_float(r[ch * 8 + 3])),
+                                             pack_bf16x2(__uint_as_float(r[ch * 8 + 4]), __uint_as_float(r[ch * 8 + 5])),
+                                             pack_bf16x2(__uint_as_float(r[ch * 8 + 6]), __uint_as_float(r[ch * 8 + 7])));
+                            }
                         }
                     }
+                    tc_fence_before();
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar[Cfg::B_OSTFULL + osb]);
+                    if (lane == 0) {
+                        mbar_arrive(&bar[Cfg::B_OEMPTY + ob]);
+                        mbar_arrive(&bar[Cfg::B_OSTFULL + osb]);
+                        if (warp == 12) LA_TRACE(31, g);
+                    }
                     if (elected) {
-                        if (mbar_wait(&bar[Cfg::B_OSTFULL + osb], (f / Cfg::OSB) & 1, abort_flag, tmo,
-                                      0x420 + osb)) {
+                        if (mbar_wait(&bar[Cfg::B_OSTFULL + osb], (f / 2) & 1, abort_flag, tmo, 0x420 + osb)) {
 #pragma unroll
                             for (int pn = 0; pn < Cfg::NPAN; ++pn)
                                 tma_store_3d(&tmO, smem + (stg - sbase) + pn * Cfg::PANEL, pn * 64,
                                              un.row0 + c * C, un.group);
                             bulk_commit_group();
-                            bulk_wait_group_read<Cfg::OSB - 1>();
-                            if (f - (Cfg::OSB - 1) >= 0)
-                                mbar_arrive(&bar[Cfg::B_OSTFREE + ((f - (Cfg::OSB - 1)) % Cfg::OSB)]);
+                            if constexpr (Cfg::PT) {
+                                // the stage returns to the producer once the store has read it
+                                bulk_wait_group_read<0>();
+                                mbar_arrive(&bar[Cfg::B_EMPTY + st_s]);
+                            } else {
+                                bulk_wait_group_read<1>();
+                                if (f >= 1) mbar_arrive(&bar[Cfg::B_OSTFREE + ((f - 1) & 1)]);
+                            }
                         }
                     }
                     ++f;
-                } else if (row >= 0 && row < nv) {
+                } else {
                     // Last, partial chunk of a sequence: plain stores of the
                     // valid rows only (the next sequence's rows follow).
-                    uint4* dst = reinterpret_cast<uint4*>(obase + (grow0 + row) * D);
+                    const bool valid = row >= 0 && row < nv;
+                    uint4* dst = reinterpret_cast<uint4*>(obase + (grow0 + (valid ? row : 0)) * D);
 #pragma unroll
-                    for (int ch = 0; ch < D / 8; ++ch)
-                        dst[ch] = make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        uint32_t r[32];
+                        tmem_ld32(tm_O + cb * 32, r);
+                        tmem_wait_ld();
+                        if (valid) {
+#pragma unroll
+                            for (int ch = 0; ch < 4; ++ch)
+                                dst[cb * 4 + ch] = make_uint4(
+                                    pack_bf16x2(__uint_as_float(r[ch * 8 + 0]), __uint_as_float(r[ch * 8 + 1])),
+                                    pack_bf16x2(__uint_as_float(r[ch * 8 + 2]), __uint_as_float(r[ch * 8 + 3])),
+                                    pack_bf16x2(__uint_as_float(r[ch * 8 + 4]), __uint_as_float(r[ch * 8 + 5])),
+                                    pack_bf16x2(__uint_as_float(r[ch * 8 + 6]), __uint_as_float(r[ch * 8 + 7])));
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar[Cfg::B_OEMPTY + ob]);
+                    if (Cfg::PT && elected) mbar_arrive(&bar[Cfg::B_EMPTY + st_s]);
                 }
             }
         }

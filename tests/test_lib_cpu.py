@@ -47,7 +47,7 @@ def test_kernel_choice():
     assert la.la_prefill_path(torch.float32, 2, 2, 4) == "simt"
     assert la.la_prefill_path(torch.bfloat16, 256, 256, 64) == "unsupported"
     assert la.la_prefill_path(torch.float32, 128, 128, 256) == "unsupported"   # tiles exceed smem
-    assert la.la_resolve_chunk(torch.bfloat16, 128, 128, 0) == 64
+    assert la.la_resolve_chunk(torch.bfloat16, 128, 128, 0) == 128
     assert la.la_resolve_chunk(torch.bfloat16, 128, 128, 96) == 96
 
 
