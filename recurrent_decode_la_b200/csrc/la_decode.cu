@@ -12,6 +12,7 @@
 // q^T S' for its columns; the partials of the rows are summed in shared
 // memory.
 #include <cuda_bf16.h>
+#include <stdlib.h>
 
 #include "la_internal.h"
 
@@ -101,6 +102,87 @@ __global__ void __launch_bounds__(kDecThreads) decode_vec_kernel(const T* __rest
     }
 }
 
+// Column-split form: the d_v columns of a unit's state are split over CB
+// CTAs, each of which owns all d_k rows of its columns, so o[j] (a sum over
+// rows of column j) needs no reduction across CTAs.  With a few hundred units
+// this still fills every SM and keeps more loads in flight per SM.  Launched
+// as a programmatic dependent of the previous kernel in the stream: a CTA may
+// start while that kernel drains, but reads nothing from global memory before
+// griddepcontrol.wait returns.
+template <typename T, int NR>
+__global__ void __launch_bounds__(kDecThreads, 4) decode_cols_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                                     const T* __restrict__ v, T* __restrict__ o,
+                                                                     float* __restrict__ state, int64_t n_units,
+                                                                     int dk, int dv, int cb_count) {
+    extern __shared__ float sm[];
+    float* qs = sm;
+    float* ks = qs + 128;
+    float* vs = ks + 128;
+    float* red = vs + 128;  // [rows per pass][cols of this CTA]
+    const int64_t u = blockIdx.x / cb_count;
+    const int cb = static_cast<int>(blockIdx.x % cb_count);
+    const int ncol = dv / cb_count;        // columns of this CTA
+    const int cbeg = cb * ncol;
+    const int cols4 = ncol >> 2;
+    const int rpp = kDecThreads / cols4;   // rows per pass
+    const int tid = threadIdx.x;
+    const int c4 = tid % cols4;
+    const int r0 = tid / cols4;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    float4* S = reinterpret_cast<float4*>(state + u * static_cast<int64_t>(dk) * dv + cbeg) + c4;
+    const int row4 = dv >> 2;  // float4 per state row
+    // first batch of this thread's rows: loads in flight before anything else
+    float4 sv[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+        const int r = r0 + i * rpp;
+        if (r < dk) sv[i] = S[r * row4];
+    }
+    for (int i = tid; i < dk; i += kDecThreads) {
+        qs[i] = dec_in<T>(q, u * dk + i);
+        ks[i] = dec_in<T>(k, u * dk + i);
+    }
+    for (int i = tid; i < ncol; i += kDecThreads) vs[i] = dec_in<T>(v, u * dv + cbeg + i);
+    __syncthreads();
+    const float4 vv = make_float4(vs[4 * c4], vs[4 * c4 + 1], vs[4 * c4 + 2], vs[4 * c4 + 3]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int rb = 0; r0 + rb * rpp < dk; rb += NR) {
+        if (rb > 0) {
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+                const int r = r0 + (rb + i) * rpp;
+                if (r < dk) sv[i] = S[r * row4];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const int r = r0 + (rb + i) * rpp;
+            if (r < dk) {
+                const float kr = ks[r], qr = qs[r];
+                float4 s4 = sv[i];
+                s4.x = fmaf(kr, vv.x, s4.x);
+                s4.y = fmaf(kr, vv.y, s4.y);
+                s4.z = fmaf(kr, vv.z, s4.z);
+                s4.w = fmaf(kr, vv.w, s4.w);
+                S[r * row4] = s4;
+                acc.x = fmaf(qr, s4.x, acc.x);
+                acc.y = fmaf(qr, s4.y, acc.y);
+                acc.z = fmaf(qr, s4.z, acc.z);
+                acc.w = fmaf(qr, s4.w, acc.w);
+            }
+        }
+    }
+    reinterpret_cast<float4*>(red + r0 * ncol)[c4] = acc;
+    __syncthreads();
+    for (int n = tid; n < ncol; n += kDecThreads) {
+        float sum = 0.f;
+        for (int rr = 0; rr < rpp && rr < dk; ++rr) sum += red[rr * ncol + n];
+        dec_out<T>(o, u * dv + cbeg + n, sum);
+    }
+}
+
 // Scalar form for any d_k, d_v <= 128 and any alignment.
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads) decode_scalar_kernel(const T* __restrict__ q, const T* __restrict__ k,
@@ -143,9 +225,48 @@ __global__ void __launch_bounds__(kDecThreads) decode_scalar_kernel(const T* __r
     }
 }
 
+static int env_int(const char* name, int dflt) {
+    const char* e = getenv(name);
+    return e && *e ? atoi(e) : dflt;
+}
+
+template <typename T>
+static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* state, int64_t n_units, int dk,
+                               int dv, int cb, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_units * cb), 1, 1);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = sizeof(float) * (3 * 128 + 1024);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = env_int("LINATTN_DECODE_PDL", 1) ? 1 : 0;
+    // rows per thread held in registers at once (batches of up to 4): few
+    // registers, so four 256-thread CTAs stay resident per SM
+    const int rpp = kDecThreads / (dv / (4 * cb));
+    const int need = (dk + rpp - 1) / rpp;
+    if (need <= 1) return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 1>, q, k, v, o, state, n_units, dk, dv, cb);
+    if (need <= 2) return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 2>, q, k, v, o, state, n_units, dk, dv, cb);
+    return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 4>, q, k, v, o, state, n_units, dk, dv, cb);
+}
+
+// Column blocks per unit: enough CTAs to cover the SMs about three times,
+// each block a whole number of float4 columns, at most 16 rows per thread.
+static int decode_col_blocks(int64_t n_units, int num_sms, int dk, int dv) {
+    auto ok = [&](int cb) {
+        if (dv % (4 * cb) != 0) return false;
+        const int cols4 = dv / (4 * cb);
+        return kDecThreads % cols4 == 0;
+    };
+    int cb = 1;
+    while (cb < 8 && n_units * cb < 3LL * num_sms && ok(cb * 2)) cb *= 2;
+    return ok(cb) ? cb : 0;
+}
+
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* state,
                           int dtype, int64_t n_units, int dk, int dv, int num_sms, cudaStream_t s) {
-    (void)num_sms;
     if (n_units <= 0) return cudaSuccess;
     const unsigned grid = static_cast<unsigned>(n_units < 2147483647 ? n_units : 2147483647);
     const size_t smem = sizeof(float) * (3 * 128 + 1024);
@@ -153,6 +274,25 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     const bool vec = (dv % 4 == 0) && cols4 > 0 && (kDecThreads % cols4 == 0) &&
                      (reinterpret_cast<uintptr_t>(state) % 16 == 0) &&
                      ((dk + (kDecThreads / cols4) - 1) / (kDecThreads / cols4) <= kDecMaxRowsPerThread);
+    // 2^31 CTAs at most; the cluster form needs n_units * CL of them.
+    // LINATTN_DECODE_COLBLOCKS overrides the column split (0 = one CTA per unit
+    // without a programmatic launch).
+    int cb = (vec && n_units <= (1LL << 27)) ? decode_col_blocks(n_units, num_sms, dk, dv) : 0;
+    const int force = env_int("LINATTN_DECODE_COLBLOCKS", -1);
+    if (vec && force >= 0) cb = force;
+    if (cb > 0 && (dv % (4 * cb) != 0 || kDecThreads % (dv / (4 * cb)) != 0)) cb = 0;
+    if (cb > 0) {
+        cudaError_t e;
+        if (dtype == 0)
+            e = launch_cols<float>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                   static_cast<const float*>(v), static_cast<float*>(o), state, n_units, dk, dv, cb, s);
+        else
+            e = launch_cols<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                           static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state,
+                                           n_units, dk, dv, cb, s);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     if (dtype == 0) {
         const float *qq = static_cast<const float*>(q), *kk = static_cast<const float*>(k),
                     *vv = static_cast<const float*>(v);
