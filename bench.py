@@ -279,12 +279,14 @@ def run_ours(args, wl, world, rank, local):
     od = torch.empty_like(dv)
     state = torch.empty(units, d, d, dtype=torch.float32, device=dev)
     path = la.la_prefill_path(dt, d, d, chunk, q, k, v, o)
+    ws_bytes = la.la_prefill_workspace_size(dt, B, H, T, d, d, 0, chunk)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
 
     stream = torch.cuda.Stream(device=dev)
 
     def prefill_phase(s):
         la.la_state_init(state, None, stream=s)
-        la.la_prefill(q, k, v, o, state, chunk=chunk, stream=s)
+        la.la_prefill(q, k, v, o, state, chunk=chunk, workspace=ws, stream=s)
 
     def decode_phase(s):
         for i in range(dsteps):
@@ -361,7 +363,7 @@ def run_ours(args, wl, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": B, "H": H, "T": T, "d_k": d, "d_v": d, "chunk": chunk,
-                   "decode_steps": dsteps, "prefill_kernel": path,
+                   "decode_steps": dsteps, "prefill_kernel": path, "workspace_bytes": ws_bytes,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (q/k/v %.0f MB per rank); decode state is the "
                          "prefill's output and stays L2-resident within a step" % (3 * q.numel() * elem / 1e6)},
@@ -392,7 +394,7 @@ def run_ours(args, wl, world, rank, local):
 
     if args.sweep_chunks:
         result["chunk_sweep"] = chunk_sweep(la, torch, stream, q, k, v, o, state, wl,
-                                            [int(c) for c in args.sweep_chunks.split(",")], peaks)
+                                            [int(c) for c in args.sweep_chunks.split(",")], peaks, dev)
 
     if not args.no_cold_decode and dsteps:
         result["decode_cold"] = cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_src)
@@ -412,7 +414,7 @@ def run_ours(args, wl, world, rank, local):
     return 0
 
 
-def chunk_sweep(la, torch, stream, q, k, v, o, state, wl, chunks, peaks):
+def chunk_sweep(la, torch, stream, q, k, v, o, state, wl, chunks, peaks, dev):
     """Prefill alone at several chunk sizes (C never changes the result, only
     the cost): CUDA-event time of one launch, median of 20 after 3 warm-ups."""
     out = {}
@@ -421,13 +423,15 @@ def chunk_sweep(la, torch, stream, q, k, v, o, state, wl, chunks, peaks):
     byts = prefill_bytes(units, wl.T, d, d, elem)
     for c in chunks:
         path = la.la_prefill_path(wl.torch_dtype, d, d, c, q, k, v, o)
+        nb = la.la_prefill_workspace_size(wl.torch_dtype, wl.B, wl.H, wl.T, d, d, 0, c)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
         ts = []
         with torch.cuda.stream(stream):
             for i in range(23):
                 la.la_state_init(state, None, stream=stream)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                la.la_prefill(q, k, v, o, state, chunk=c, stream=stream)
+                la.la_prefill(q, k, v, o, state, chunk=c, workspace=ws, stream=stream)
                 e1.record(stream)
                 e1.synchronize()
                 if i >= 3:
@@ -494,12 +498,14 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
     o = torch.empty_like(dev_bufs[2])
     od = torch.empty_like(dev_bufs[5])
     st = torch.empty(B * H, d, d, dtype=torch.float32, device=dev)
+    nb = la.la_prefill_workspace_size(wl.torch_dtype, B, H, T, d, d, 0, chunk)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
 
     def step():
         for h, dbuf in zip(pins, dev_bufs):
             dbuf.copy_(h, non_blocking=True)
         la.la_state_init(st, None, stream=stream)
-        la.la_prefill(dev_bufs[0], dev_bufs[1], dev_bufs[2], o, st, chunk=chunk, stream=stream)
+        la.la_prefill(dev_bufs[0], dev_bufs[1], dev_bufs[2], o, st, chunk=chunk, workspace=ws, stream=stream)
         for i in range(dsteps):
             la.la_decode_step(dev_bufs[3][i], dev_bufs[4][i], dev_bufs[5][i], od[i], st, stream=stream)
         o_h.copy_(o, non_blocking=True)

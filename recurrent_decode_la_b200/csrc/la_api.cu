@@ -99,6 +99,46 @@ struct TraceBuf {
 };
 TraceBuf g_trace;
 
+// Intra-sequence split plan (dense bf16 tensor-core input with fewer units
+// than SMs): seg_count segments per unit run as separate work items, each
+// starting from S_0 plus the K^T V sums of the sub-segments before it.
+struct SplitPlan {
+    int seg_count = 1;
+    int64_t seg_len = 0;
+    int64_t sub_len = 0;
+    int subs_per_seg = 0;
+    int subs_per_unit = 0;
+    size_t bytes = 0;
+};
+
+SplitPlan plan_split(int64_t n_units, int64_t T, int dk, int dv, int chunk, int sms) {
+    SplitPlan sp;
+    sp.seg_len = T;
+    const char* e = getenv("LINATTN_SPLIT");
+    if (e && e[0] == '0') return sp;
+    if (n_units <= 0 || T <= 0) return sp;
+    const int64_t nch = (T + chunk - 1) / chunk;
+    int64_t P = sms / n_units;
+    if (P > 8) P = 8;
+    if (P > nch / 4) P = nch / 4;  // at least four chunks per segment
+    if (P < 2) return sp;
+    const int64_t seg_chunks = (nch + P - 1) / P;
+    const int64_t seg_len = seg_chunks * chunk;
+    P = (T + seg_len - 1) / seg_len;
+    if (P < 2) return sp;
+    // sub-segments: enough work items for the first pass to cover the SMs
+    const int64_t base_items = n_units * (P - 1);
+    int k = 1;
+    while (k < 16 && base_items * k < 3LL * sms && seg_chunks % (2 * k) == 0) k *= 2;
+    sp.seg_count = static_cast<int>(P);
+    sp.seg_len = seg_len;
+    sp.sub_len = seg_len / k;
+    sp.subs_per_seg = k;
+    sp.subs_per_unit = static_cast<int>((P - 1) * k);
+    sp.bytes = static_cast<size_t>(n_units) * sp.subs_per_unit * dk * dv * sizeof(float);
+    return sp;
+}
+
 enum Path { kTc, kSimt, kUnsupported };
 
 Path choose_path(la_dtype dtype, int dk, int dv, int chunk, const void* q, const void* k, const void* v,
@@ -155,14 +195,18 @@ la_status la_state_init(float* state, const float* src, int64_t n_units, int d_k
 
 size_t la_prefill_workspace_size(la_dtype dtype, int B, int H, int64_t T, int d_k, int d_v, int num_seqs,
                                  int chunk) {
-    (void)dtype; (void)B; (void)H; (void)T; (void)d_k; (void)d_v; (void)num_seqs; (void)chunk;
-    return 0;
+    // Only dense bf16 input on the tensor-core path is split; packed input
+    // (num_seqs > 0) never is.
+    if (num_seqs > 0 || B <= 0 || H <= 0 || T <= 0) return 0;
+    const int c = la_resolve_chunk(dtype, d_k, d_v, chunk);
+    if (!(dtype == LA_BF16 && d_k == d_v && prefill_tc_supported(d_k, c))) return 0;
+    return plan_split(static_cast<int64_t>(B) * H, T, d_k, d_v, c, current_sm_count()).bytes;
 }
 
 la_status la_prefill(const void* q, const void* k, const void* v, void* o, float* state, la_dtype dtype, int B,
                      int H, int64_t T, int d_k, int d_v, const int32_t* cu_seqlens, int num_seqs,
                      int64_t max_seqlen, int chunk, void* workspace, size_t workspace_bytes, void* stream) {
-    (void)max_seqlen; (void)workspace; (void)workspace_bytes;
+    (void)max_seqlen;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || T < 0 || d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
     if (T > 0x7fffffffLL) return LA_ERR_UNSUPPORTED;
@@ -194,6 +238,12 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     p.cu = cu_seqlens;
     p.chunk = c;
     p.timeout_ns = wait_timeout_ns();
+    p.seg_count = 1;
+    p.seg_len = T;
+    p.sub_len = 0;
+    p.subs_per_seg = 0;
+    p.subs_per_unit = 0;
+    p.sub_states = nullptr;
     p.trace = g_trace.buf;
     p.trace_count = g_trace.count;
     p.trace_cap = g_trace.cap;
@@ -206,6 +256,21 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
             !encode_bf16_map(&tv, v, d_v, T, groups, c) || !encode_bf16_map(&to, o, d_v, T, groups, c)) {
             snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
             return LA_ERR_CUDA;
+        }
+        // Few long sequences: split each one so that every SM gets work, when
+        // the caller provided the workspace la_prefill_workspace_size asks for.
+        if (!cu_seqlens) {
+            const SplitPlan sp = plan_split(n_units, T, d_k, d_v, c, sms);
+            if (sp.seg_count > 1 && workspace && workspace_bytes >= sp.bytes && aligned16(workspace)) {
+                p.seg_count = sp.seg_count;
+                p.seg_len = sp.seg_len;
+                p.sub_len = sp.sub_len;
+                p.subs_per_seg = sp.subs_per_seg;
+                p.subs_per_unit = sp.subs_per_unit;
+                p.sub_states = static_cast<const float*>(workspace);
+                e = launch_subsegment_states(p, tk, tv, static_cast<float*>(workspace), sms, s);
+                if (e != cudaSuccess) return cuda_fail(e);
+            }
         }
         e = launch_prefill_tc(p, tq, tk, tv, to, sms, s);
     } else {

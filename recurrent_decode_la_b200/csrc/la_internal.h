@@ -26,6 +26,18 @@ struct PrefillProblem {
     const int32_t* cu;  // nullptr for dense input
     int chunk;
     uint64_t timeout_ns;
+    // Intra-sequence split (dense input only; seg_count = 1 means none).
+    // Work item i is segment i % seg_count of unit i / seg_count: rows
+    // [s * seg_len, min((s + 1) * seg_len, rows_per_group)).  Segment s starts
+    // from S_0 plus the K^T V sums of the first s * subs_per_seg sub-segments
+    // (sub_len rows each) in sub_states [units][subs_per_unit][dk][dv]; only
+    // the last segment writes S_T.
+    int seg_count;
+    int64_t seg_len;
+    int64_t sub_len;
+    int subs_per_seg;
+    int subs_per_unit;
+    const float* sub_states;
     // Event trace of CTA 0 (builds with LINATTN_TRACE only; nullptr otherwise).
     unsigned long long* trace;
     unsigned int* trace_count;
@@ -40,6 +52,12 @@ bool prefill_tc_supported(int D, int chunk);
 cudaError_t launch_prefill_tc(const PrefillProblem& p, const CUtensorMap& tq,
                               const CUtensorMap& tk, const CUtensorMap& tv,
                               const CUtensorMap& to, int num_sms, cudaStream_t s);
+
+// Sub-segment states for the intra-sequence split: sub_states[u][j] =
+// K^T V over rows [j * sub_len, (j + 1) * sub_len) of unit u, for
+// j < subs_per_unit (tensor cores, bf16 in, fp32 out).
+cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                     float* sub_states, int num_sms, cudaStream_t s);
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* state,
                           int dtype, int64_t n_units, int dk, int dv, int num_sms,

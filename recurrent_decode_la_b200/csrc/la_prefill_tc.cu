@@ -101,21 +101,32 @@ struct TcCfg {
 };
 
 struct Unit {
-    int group;
-    int row0;
-    int len;
+    int group;     // TMA group coordinate (b*H + h dense, h packed)
+    int row0;      // first row of this work item
+    int len;       // rows of this work item
+    int64_t unit;  // state index
+    int seg;       // segment of the unit (0 without a split)
+    bool last;     // the item that writes S_T
 };
 
-// Rows of unit u.  A packed sequence whose offsets are out of range or
-// decreasing is treated as empty (its state is left untouched).
-__device__ __forceinline__ Unit get_unit(const PrefillProblem& p, int64_t u) {
-    if (p.cu == nullptr) return {static_cast<int>(u), 0, static_cast<int>(p.rows_per_group)};
-    const int n = static_cast<int>(u / p.H);
-    const int h = static_cast<int>(u % p.H);
+// Work item i.  Without a split an item is a unit.  A packed sequence whose
+// offsets are out of range or decreasing is treated as empty (its state is
+// left untouched).
+__device__ __forceinline__ Unit get_unit(const PrefillProblem& p, int64_t i) {
+    if (p.cu == nullptr) {
+        const int64_t u = i / p.seg_count;
+        const int seg = static_cast<int>(i % p.seg_count);
+        const int64_t r0 = seg * p.seg_len;
+        const int64_t r1 = min(r0 + p.seg_len, p.rows_per_group);
+        return {static_cast<int>(u), static_cast<int>(r0), static_cast<int>(r1 - r0), u, seg,
+                seg == p.seg_count - 1};
+    }
+    const int n = static_cast<int>(i / p.H);
+    const int h = static_cast<int>(i % p.H);
     const int a = p.cu[n];
     const int b = p.cu[n + 1];
-    if (a < 0 || b < a || static_cast<int64_t>(b) > p.rows_per_group) return {h, 0, 0};
-    return {h, a, b - a};
+    if (a < 0 || b < a || static_cast<int64_t>(b) > p.rows_per_group) return {h, 0, 0, i, 0, true};
+    return {h, a, b - a, i, 0, true};
 }
 
 // Accumulator row held by lane `lane` of a warp reading its TMEM
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(512, 1)
             int64_t last_g[Cfg::NS];
             for (int s = 0; s < Cfg::NS; ++s) last_g[s] = -1;
             bool ok = true;
-            for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+            for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
                 const Unit un = get_unit(p, u);
                 const int nch = (un.len + C - 1) / C;
                 for (int c = 0; c < nch; ++c, ++g) {
@@ -265,7 +276,7 @@ __global__ void __launch_bounds__(512, 1)
         auto first = [&](Cursor& k) {
             k.g = 0;
             k.c = 0;
-            for (k.u = blockIdx.x; k.u < p.n_units; k.u += gridDim.x) {
+            for (k.u = blockIdx.x; k.u < p.n_units * p.seg_count; k.u += gridDim.x) {
                 const Unit un = get_unit(p, k.u);
                 k.nch = (un.len + C - 1) / C;
                 if (k.nch > 0) {
@@ -284,7 +295,7 @@ __global__ void __launch_bounds__(512, 1)
                 return;
             }
             k.c = 0;
-            for (k.u += gridDim.x; k.u < p.n_units; k.u += gridDim.x) {
+            for (k.u += gridDim.x; k.u < p.n_units * p.seg_count; k.u += gridDim.x) {
                 const Unit un = get_unit(p, k.u);
                 k.nch = (un.len + C - 1) / C;
                 if (k.nch > 0) {
@@ -477,7 +488,7 @@ __global__ void __launch_bounds__(512, 1)
         const int rowA = acc_row<C>(sub, lane);  // score / P row
         int64_t g = 0;
         bool ok = true;
-        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+        for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
             const Unit un = get_unit(p, u);
             const int nch = (un.len + C - 1) / C;
             for (int c = 0; c < nch; ++c, ++g) {
@@ -559,12 +570,18 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t tm_S = tmem + Cfg::TM_S + lane_off;
         int64_t g = 0;
         bool ok = true;
-        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+        for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
             const Unit un = get_unit(p, u);
             const int nch = (un.len + C - 1) / C;
             if (nch == 0) continue;
-            float* st_row = p.state + u * static_cast<int64_t>(D) * D +
+            float* st_row = p.state + un.unit * static_cast<int64_t>(D) * D +
                             static_cast<int64_t>(rowS < 0 ? 0 : rowS) * D;
+            // a segment after the first starts from S_0 plus the K^T V sums of
+            // every sub-segment before it
+            const int nsub = un.seg * p.subs_per_seg;
+            const float* sub_row = nsub > 0 ? p.sub_states + un.unit * static_cast<int64_t>(p.subs_per_unit) * D * D +
+                                                  static_cast<int64_t>(rowS < 0 ? 0 : rowS) * D
+                                            : nullptr;
             // ---- unit start: S_0 into TMEM (fp32) and into the bf16 operand
             if (g > 0 && !mbar_wait_warp(&bar[Cfg::B_SBEMPTY], (g - 1) & 1, abort_flag, tmo, 0x300)) {
                 ok = false;
@@ -577,7 +594,15 @@ __global__ void __launch_bounds__(512, 1)
                     const float4* src = reinterpret_cast<const float4*>(st_row + cb * 32);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const float4 f = src[i];
+                        float4 f = src[i];
+                        for (int j = 0; j < nsub; ++j) {
+                            const float4 d4 = reinterpret_cast<const float4*>(
+                                sub_row + static_cast<int64_t>(j) * D * D + cb * 32)[i];
+                            f.x += d4.x;
+                            f.y += d4.y;
+                            f.z += d4.z;
+                            f.w += d4.w;
+                        }
                         r[4 * i + 0] = __float_as_uint(f.x);
                         r[4 * i + 1] = __float_as_uint(f.y);
                         r[4 * i + 2] = __float_as_uint(f.z);
@@ -626,7 +651,7 @@ __global__ void __launch_bounds__(512, 1)
                     uint32_t r[32];
                     tmem_ld32(tm_S + cb * 32, r);
                     tmem_wait_ld();
-                    if (last && rowS >= 0) {
+                    if (last && un.last && rowS >= 0) {
                         float4* dst = reinterpret_cast<float4*>(st_row + cb * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
@@ -671,7 +696,7 @@ __global__ void __launch_bounds__(512, 1)
         uint16_t* obase = static_cast<uint16_t*>(p.o);
         int64_t g = 0, f = 0;
         bool ok = true;
-        for (int64_t u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+        for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
             const Unit un = get_unit(p, u);
             const int nch = (un.len + C - 1) / C;
             for (int c = 0; c < nch; ++c, ++g) {
@@ -780,6 +805,210 @@ __global__ void __launch_bounds__(512, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Sub-segment states for the intra-sequence split.  Because the state is a
+// plain sum (S_t = S_0 + sum over j <= t of k_j v_j^T), the state a segment
+// starts from is S_0 plus the K^T V sums of the segments before it; this
+// kernel computes those sums for sub-segments of sub_len rows, on the tensor
+// cores, one sub-segment per work item:
+//   warp 0      TMA producer (K and V chunk tiles, NS-deep ring)
+//   warp 1      MMA issuer: S_j += K_c^T V_c, two TMEM accumulators so the
+//               next sub-segment accumulates while the last one is written
+//   warps 2-5   epilogue: TMEM -> fp32 rows of sub_states
+// Waits are bounded as in the prefill kernel.
+// ---------------------------------------------------------------------------
+template <int C, int D>
+struct KvCfg {
+    static constexpr int kThreads = 192;
+    static constexpr int PANEL = C * 128;
+    static constexpr int NPAN = D / 64;
+    static constexpr int TILE = C * D * 2;
+    static constexpr int STAGE = 2 * TILE;  // K, V
+    static constexpr int NS = (3 * STAGE <= 200 * 1024) ? 3 : 2;
+    static constexpr int OFF_BAR = NS * STAGE;
+    static constexpr int SMEM = OFF_BAR + 32 * 8 + 16 + 1024;
+    static constexpr int TM_COLS = (2 * D <= 128) ? 128 : 256;
+    static constexpr int B_FULL = 0, B_EMPTY = 8, B_AFULL = 16, B_AEMPTY = 18, B_DONE = 20;
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <int C, int D>
+__global__ void __launch_bounds__(192, 1)
+    subsegment_states_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                             const PrefillProblem p, float* __restrict__ sub_states) {
+    using Cfg = KvCfg<C, D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_BAR + 32 * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_BAR + 32 * 8 + 4);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint64_t tmo = p.timeout_ns;
+    const int64_t n_items = p.n_units * p.subs_per_unit;
+    const int nch = static_cast<int>((p.sub_len + C - 1) / C);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::NS; ++s) {
+            mbar_init(&bar[Cfg::B_FULL + s], 1);
+            mbar_init(&bar[Cfg::B_EMPTY + s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar[Cfg::B_AFULL + b], 1);
+            mbar_init(&bar[Cfg::B_AEMPTY + b], 4);
+        }
+        mbar_init(&bar[Cfg::B_DONE], 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base_slot, Cfg::TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_slot;
+    const uint32_t sbase = smem_u32(smem);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int64_t g = 0;
+            int64_t last_g[Cfg::NS];
+            for (int s = 0; s < Cfg::NS; ++s) last_g[s] = -1;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+                const int64_t u = it / p.subs_per_unit;
+                const int64_t j = it % p.subs_per_unit;
+                for (int c = 0; c < nch; ++c, ++g) {
+                    const int s = static_cast<int>(g % Cfg::NS);
+                    if (g >= Cfg::NS && !mbar_wait(&bar[Cfg::B_EMPTY + s], ((g / Cfg::NS) + 1) & 1, abort_flag,
+                                                   tmo, 0x500 + s)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bar[Cfg::B_FULL + s], Cfg::STAGE);
+                    const int row = static_cast<int>(j * p.sub_len) + c * C;
+#pragma unroll
+                    for (int pn = 0; pn < Cfg::NPAN; ++pn) {
+                        tma_load_3d(smem + s * Cfg::STAGE + pn * Cfg::PANEL, &tmK, &bar[Cfg::B_FULL + s], pn * 64,
+                                    row, static_cast<int>(u));
+                        tma_load_3d(smem + s * Cfg::STAGE + Cfg::TILE + pn * Cfg::PANEL, &tmV, &bar[Cfg::B_FULL + s],
+                                    pn * 64, row, static_cast<int>(u));
+                    }
+                    last_g[s] = g;
+                }
+            }
+            if (!ok || *abort_flag) {
+                for (int s = 0; s < Cfg::NS; ++s)
+                    if (last_g[s] >= 0) mbar_wait_drain(&bar[Cfg::B_FULL + s], (last_g[s] / Cfg::NS) & 1, tmo);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t kIdKV = idesc_bf16_f32(D, D, true, true);
+            int64_t g = 0, local = 0;
+            bool ok = true, issued = false;
+            for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++local) {
+                const int b = static_cast<int>(local & 1);
+                if (local >= 2 && !mbar_wait(&bar[Cfg::B_AEMPTY + b], ((local >> 1) + 1) & 1, abort_flag, tmo,
+                                             0x510 + b)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t tm_S = tmem + b * D;
+                for (int c = 0; c < nch; ++c, ++g) {
+                    const int s = static_cast<int>(g % Cfg::NS);
+                    if (!mbar_wait(&bar[Cfg::B_FULL + s], (g / Cfg::NS) & 1, abort_flag, tmo, 0x520 + s)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t kb = sbase + s * Cfg::STAGE, vb = kb + Cfg::TILE;
+#pragma unroll
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_bf16_ss(tm_S, sdesc_sw128(kb + ks * 2048, Cfg::PANEL, 1024),
+                                    sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024), kIdKV, (c > 0 || ks > 0) ? 1u : 0u);
+                    mma_commit(&bar[Cfg::B_EMPTY + s]);
+                    issued = true;
+                }
+                if (ok) mma_commit(&bar[Cfg::B_AFULL + b]);
+            }
+            if (issued) {
+                mma_commit(&bar[Cfg::B_DONE]);
+                mbar_wait_drain(&bar[Cfg::B_DONE], 0, tmo);
+            }
+        }
+        __syncwarp();
+    } else {
+        // epilogue warps 2..5 cover TMEM sub-partitions 2, 3, 0, 1
+        const int sub = warp & 3;
+        const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+        const int row = acc_row<D>(sub, lane);
+        int64_t local = 0;
+        for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, ++local) {
+            const int b = static_cast<int>(local & 1);
+            if (!mbar_wait_warp(&bar[Cfg::B_AFULL + b], (local >> 1) & 1, abort_flag, tmo, 0x530 + b)) break;
+            tc_fence_after();
+            float* dst = sub_states + it * static_cast<int64_t>(D) * D + static_cast<int64_t>(row < 0 ? 0 : row) * D;
+#pragma unroll
+            for (int cb = 0; cb < D / 32; ++cb) {
+                uint32_t r[32];
+                tmem_ld32(tmem + b * D + lane_off + cb * 32, r);
+                tmem_wait_ld();
+                if (row >= 0) {
+                    float4* d4 = reinterpret_cast<float4*>(dst + cb * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[Cfg::B_AEMPTY + b]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::TM_COLS);
+    }
+}
+
+template <int C, int D>
+static cudaError_t launch_sub_impl(const PrefillProblem& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                   float* sub_states, int num_sms, cudaStream_t s) {
+    using Cfg = KvCfg<C, D>;
+    auto kern = subsegment_states_kernel<C, D>;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    const int64_t items = p.n_units * p.subs_per_unit;
+    const int64_t grid = items < num_sms ? items : num_sms;
+    if (grid < 1) return cudaSuccess;
+    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::SMEM, s>>>(tk, tv, p, sub_states);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                     float* sub_states, int num_sms, cudaStream_t s) {
+    if (p.dk == 64 && p.chunk == 64) return launch_sub_impl<64, 64>(p, tk, tv, sub_states, num_sms, s);
+    if (p.dk == 128 && p.chunk == 64) return launch_sub_impl<64, 128>(p, tk, tv, sub_states, num_sms, s);
+    if (p.dk == 64 && p.chunk == 128) return launch_sub_impl<128, 64>(p, tk, tv, sub_states, num_sms, s);
+    if (p.dk == 128 && p.chunk == 128) return launch_sub_impl<128, 128>(p, tk, tv, sub_states, num_sms, s);
+    return cudaErrorInvalidValue;
+}
+
 bool prefill_tc_supported(int D, int chunk) {
     return (D == 64 || D == 128) && (chunk == 64 || chunk == 128);
 }
@@ -801,7 +1030,8 @@ static cudaError_t launch_tc_impl(const PrefillProblem& p, const CUtensorMap& tq
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    int64_t grid = p.n_units < num_sms ? p.n_units : num_sms;
+    const int64_t items = p.n_units * p.seg_count;
+    int64_t grid = items < num_sms ? items : num_sms;
     if (grid < 1) return cudaSuccess;
     kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::SMEM, s>>>(tq, tk, tv, to, p);
     return cudaGetLastError();

@@ -28,8 +28,9 @@ def nerr(x, ref) -> float:
     return float(diff / scale) if scale > 0 else float(diff)
 
 
-def gpu_prefill(q, k, v, S0=None, cu=None, chunk=0, max_seqlen=0):
-    """Copy CPU tensors to the GPU, run la_prefill, return (O, S_T) on the GPU."""
+def gpu_prefill(q, k, v, S0=None, cu=None, chunk=0, max_seqlen=0, workspace=True):
+    """Copy CPU tensors to the GPU, run la_prefill (with the workspace the
+    library asks for, unless workspace=False), return (O, S_T) on the GPU."""
     dev = torch.device("cuda")
     qd, kd, vd = (x.to(dev).contiguous() for x in (q, k, v))
     o = torch.empty_like(vd)
@@ -39,7 +40,13 @@ def gpu_prefill(q, k, v, S0=None, cu=None, chunk=0, max_seqlen=0):
     st = torch.empty(units, dk, dv, dtype=torch.float32, device=dev)
     la.la_state_init(st, None if S0 is None else S0.reshape(units, dk, dv).to(dev).float().contiguous())
     cud = cu.to(dev) if cu is not None else None
-    la.la_prefill(qd, kd, vd, o, st, cu_seqlens=cud, max_seqlen=max_seqlen, chunk=chunk)
+    ws = None
+    if workspace:
+        nbytes = la.la_prefill_workspace_size(q.dtype, B, H, T, dk, dv,
+                                              0 if cu is None else cu.numel() - 1, chunk)
+        if nbytes:
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    la.la_prefill(qd, kd, vd, o, st, cu_seqlens=cud, max_seqlen=max_seqlen, chunk=chunk, workspace=ws)
     assert la.la_device_status() == la.LA_OK
     return o, st
 

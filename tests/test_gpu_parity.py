@@ -101,6 +101,24 @@ def test_tc_prefill_random_state(d, chunk, T):
     assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
 
 
+@pytest.mark.parametrize("B,H,T,d,chunk", [(1, 4, 4096, 128, 128), (1, 2, 2000, 128, 64),
+                                           (2, 3, 1111, 64, 128), (1, 1, 8192, 64, 64)])
+def test_intra_sequence_split(B, H, T, d, chunk):
+    """Few units: each sequence is split into segments that start from S_0 plus
+    the K^T V sums of the earlier sub-segments.  Same result as no split."""
+    ws = la.la_prefill_workspace_size(torch.bfloat16, B, H, T, d, d, 0, chunk)
+    assert ws > 0
+    q, k, v = inputs.random_qkv(T + d, B, H, T, d, d, dtype=torch.bfloat16)
+    S0 = torch.from_numpy(np.random.default_rng(T).standard_normal((B, H, d, d)).astype(np.float32)) * 0.05
+    O_ref, S_ref = ora.recurrent(q, k, v, S0)
+    o, S = gpu_prefill(q, k, v, S0=S0, chunk=chunk)
+    assert nerr(o, O_ref) <= BF16_TOL
+    assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
+    o2, S2 = gpu_prefill(q, k, v, S0=S0, chunk=chunk, workspace=False)
+    assert nerr(o2, O_ref) <= BF16_TOL
+    assert nerr(S2.reshape(S_ref.shape), S_ref) <= BF16_TOL
+
+
 def test_tc_vs_simt_same_inputs():
     """Two kernels, two chunk sizes, one result (chunking never changes it)."""
     q, k, v = inputs.random_qkv(3, 1, 4, 200, 64, 64, dtype=torch.bfloat16)

@@ -68,7 +68,11 @@ def test_argument_checks_before_any_launch(lib):
     assert lib.la_prefill(None, None, None, None, None, 1, 0, 4, 8, 64, 64, None, 0, 0, 64, None, 0, None) == la.LA_OK
     assert lib.la_prefill(None, None, None, None, None, 1, 1, 4, 0, 64, 64, None, 0, 0, 64, None, 0, None) == la.LA_OK
     assert lib.la_state_init(None, None, 0, 8, 8, None) == la.LA_OK
-    assert lib.la_prefill_workspace_size(1, 8, 16, 8192, 128, 128, 0, 64) == 0
+    # the intra-sequence split needs workspace only for few, long, dense units
+    assert lib.la_prefill_workspace_size(1, 8, 16, 8192, 128, 128, 0, 128) == 0
+    assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 0, 128) > 0
+    assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 64, 128) == 0   # packed: never split
+    assert lib.la_prefill_workspace_size(0, 1, 32, 131072, 128, 128, 0, 128) == 0    # fp32: CUDA-core path
 
 
 def test_binding_rejects_cpu_tensors():
