@@ -98,6 +98,36 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o,
 size_t la_prefill_workspace_size(la_dtype dtype, int B, int H, int64_t T,
                                  int d_k, int d_v, int num_seqs, int chunk);
 
+/* Size of the library's own static scratch buffer used by la_prefill_noalloc
+ * (64 MiB, held on every GPU that loads the library until the process exits). */
+#define LA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* la_prefill for callers that cannot allocate device memory.  The slides have
+ * no counterpart to this entry point; it exists for callers that run inside
+ * an engine which owns every byte of device memory (a serving runtime with a
+ * fixed memory plan, a plugin living inside another framework's caching
+ * allocator) or on a path where a cudaMalloc would synchronise the device.
+ * Same arguments and results as la_prefill, without workspace: the scratch
+ * that la_prefill would take from the caller (la_prefill_workspace_size
+ * bytes) comes from a static device buffer of LA_NOALLOC_SCRATCH_BYTES inside
+ * the library.  Nothing is allocated or freed, by this call or any library it
+ * calls.
+ *   - The first call on a device looks up that device's address of the
+ *     buffer; make that first call before any stream capture.
+ *   - Every call on a device shares the one buffer, and calls that overlap
+ *     on the GPU (different streams, no ordering between them) race on it.
+ *     Every byte a call reads from the buffer was written earlier in the same
+ *     call, so nothing needs clearing between calls.
+ *   - A request whose scratch would exceed LA_NOALLOC_SCRATCH_BYTES returns
+ *     LA_ERR_UNSUPPORTED before launching anything; la_last_cuda_error()
+ *     then states the bytes needed and the bytes available.
+ * Other errors as for la_prefill. */
+la_status la_prefill_noalloc(const void* q, const void* k, const void* v,
+                             void* o, float* state, la_dtype dtype, int B,
+                             int H, int64_t T, int d_k, int d_v,
+                             const int32_t* cu_seqlens, int num_seqs,
+                             int64_t max_seqlen, int chunk, void* stream);
+
 /* One decode token for every unit ("Prefill and decode", 1x1 triangle):
  *   S' = S + k v^T, o = q^T S' (= q^T S + (q.k) v).
  *   q, k: [B, H, d_k]; v, o: [B, H, d_v] in `dtype`; state [B*H][d_k][d_v]

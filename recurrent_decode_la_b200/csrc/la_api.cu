@@ -12,6 +12,11 @@
 #include "la_device.cuh"
 #include "la_internal.h"
 
+// Scratch of la_prefill_noalloc: a static device buffer, so that entry point
+// allocates nothing.  In host code this name is only a stand-in for the
+// symbol; the device address comes from cudaGetSymbolAddress (per device).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
+
 namespace la {
 
 __device__ unsigned int g_error_word[2];
@@ -303,6 +308,44 @@ la_status la_debug_set_trace(unsigned long long* buf, unsigned int* count, unsig
     return LA_OK;
 }
 #endif
+
+la_status la_prefill_noalloc(const void* q, const void* k, const void* v, void* o, float* state, la_dtype dtype,
+                             int B, int H, int64_t T, int d_k, int d_v, const int32_t* cu_seqlens, int num_seqs,
+                             int64_t max_seqlen, int chunk, void* stream) {
+    // Scratch this request needs (the same amount la_prefill would take from
+    // a caller's workspace); refuse it up front when the static buffer is
+    // too small.
+    const size_t need = (B >= 0 && H >= 0 && T >= 0 && d_k > 0 && d_v > 0)
+                            ? la_prefill_workspace_size(dtype, B, H, T, d_k, d_v, cu_seqlens ? num_seqs : 0, chunk)
+                            : 0;
+    if (need > LA_NOALLOC_SCRATCH_BYTES) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                 "la_prefill_noalloc: needs %zu bytes of scratch, the static buffer holds %u", need,
+                 static_cast<unsigned>(LA_NOALLOC_SCRATCH_BYTES));
+        return LA_ERR_UNSUPPORTED;
+    }
+    void* scratch = nullptr;
+    if (need > 0) {
+        // Device address of the static buffer, looked up once per device
+        // with that device current.
+        static void* addr[64] = {nullptr};
+        static std::mutex mu;
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (dev < 0 || dev >= 64) return LA_ERR_UNSUPPORTED;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!addr[dev]) {
+            void* ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+            if (e != cudaSuccess) return cuda_fail(e);
+            addr[dev] = ptr;
+        }
+        scratch = addr[dev];
+    }
+    return la_prefill(q, k, v, o, state, dtype, B, H, T, d_k, d_v, cu_seqlens, num_seqs, max_seqlen, chunk, scratch,
+                      scratch ? static_cast<size_t>(LA_NOALLOC_SCRATCH_BYTES) : 0, stream);
+}
 
 la_status la_device_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
