@@ -249,6 +249,10 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     p.subs_per_seg = 0;
     p.subs_per_unit = 0;
     p.sub_states = nullptr;
+    {
+        const char* pf = getenv("LINATTN_PREFETCH");
+        p.prefetch = pf ? atoi(pf) : 1;  // measured best on B200 (deeper prefetch thrashes)
+    }
     p.trace = g_trace.buf;
     p.trace_count = g_trace.count;
     p.trace_cap = g_trace.cap;

@@ -38,6 +38,9 @@ struct PrefillProblem {
     int subs_per_seg;
     int subs_per_unit;
     const float* sub_states;
+    // Chunks ahead of the shared-memory load that the producer prefetches
+    // into L2 (0 = none).
+    int prefetch;
     // Event trace of CTA 0 (builds with LINATTN_TRACE only; nullptr otherwise).
     unsigned long long* trace;
     unsigned int* trace_count;

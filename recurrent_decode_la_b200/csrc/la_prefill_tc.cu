@@ -198,6 +198,14 @@ __global__ void __launch_bounds__(512, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_slot;
+#ifdef LINATTN_TRACE
+    if (p.trace && threadIdx.x == 0 && blockIdx.x < p.trace_cap / 64) {
+        p.trace[62 * (p.trace_cap / 64) + blockIdx.x] = globaltimer_ns();
+        unsigned int smid;
+        asm volatile("mov.u32 %0, %smid;" : "=r"(smid));
+        p.trace[61 * (p.trace_cap / 64) + blockIdx.x] = smid;
+    }
+#endif
 
     const uint32_t sbase = smem_u32(smem);
     auto stage_q = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE; };
@@ -239,6 +247,17 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     last_g[s] = g;
                     LA_TRACE(1, g);
+                    // L2 prefetch of the chunk kPrefetch ahead (same work item):
+                    // its shared-memory load then waits on L2, not on HBM.
+                    if (p.prefetch > 0 && c + p.prefetch < nch) {
+                        const int prow = un.row0 + (c + p.prefetch) * C;
+#pragma unroll
+                        for (int pn = 0; pn < Cfg::NPAN; ++pn) {
+                            tma_prefetch_l2_3d(&tmQ, pn * 64, prow, un.group);
+                            tma_prefetch_l2_3d(&tmK, pn * 64, prow, un.group);
+                            tma_prefetch_l2_3d(&tmV, pn * 64, prow, un.group);
+                        }
+                    }
                 }
             }
             if (!ok || *abort_flag) {
@@ -799,6 +818,10 @@ __global__ void __launch_bounds__(512, 1)
 
     tc_fence_before();
     __syncthreads();
+#ifdef LINATTN_TRACE
+    if (p.trace && threadIdx.x == 0 && blockIdx.x < p.trace_cap / 64)
+        p.trace[63 * (p.trace_cap / 64) + blockIdx.x] = globaltimer_ns();
+#endif
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::TM_COLS);
