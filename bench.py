@@ -140,6 +140,25 @@ def dist_env():
     return world, rank, local
 
 
+# ------------------------------------------------------ multi-rank plumbing --
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, steps: int, units_per_step_per_rank: float, ms_max: float) -> float:
+    """Weak scaling: every rank runs its own batch; the job's rate is all the
+    ranks' work divided by the slowest rank's time."""
+    return world * steps * units_per_step_per_rank / (ms_max * 1e-3)
+
+
 # ------------------------------------------------------ algorithmic sizes --
 
 def prefill_bytes(units, T, dk, dv, elem):
@@ -339,13 +358,10 @@ def run_ours(args, wl, world, rank, local):
     ms_total = t_start.elapsed_time(t_end)
     ms_pre = [e[0].elapsed_time(e[1]) for e in ev]
     ms_dec = [e[1].elapsed_time(e[2]) for e in ev]
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(ms_total, dev)
 
     tokens_step = B * T + B * dsteps              # sequence positions (all heads)
-    value = world * args.steps * tokens_step / (ms_total * 1e-3)
+    value = whole_job_rate(world, args.steps, tokens_step, ms_total)
     pre_ms = statistics.mean(ms_pre)
     dec_ms = statistics.mean(ms_dec) if dsteps else 0.0
     pre_bytes = prefill_bytes(units, T, d, d, elem)

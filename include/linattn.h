@@ -142,6 +142,15 @@ la_status la_decode_step(const void* q, const void* k, const void* v, void* o,
  * failed, else LA_OK. */
 la_status la_device_status(void* stream);
 
+/* Diagnostic of the failure path (no counterpart on the slides): launches
+ * one kernel whose single thread waits on a barrier that nothing completes,
+ * with the same bounded wait the prefill kernels use, limited to
+ * `timeout_ms`.  The kernel gives up, records the timeout in the device
+ * error word and returns; the next la_device_status() reports
+ * LA_ERR_TIMEOUT and clears it.  Nothing faults or hangs; the context stays
+ * usable.  Errors: LA_ERR_INVALID_ARG for timeout_ms outside (0, 10000]. */
+la_status la_selftest_wait_timeout(double timeout_ms, void* stream);
+
 /* Which kernel la_prefill would run for these arguments: "tc" (tensor
  * cores), "simt" (fp32 CUDA cores) or "unsupported".  Host only. */
 const char* la_prefill_path(la_dtype dtype, int d_k, int d_v, int chunk,

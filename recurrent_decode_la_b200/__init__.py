@@ -15,4 +15,5 @@ from .binding import (  # noqa: F401
     LA_F32, LA_BF16, LinAttnError, lib_path, load_library,
     la_state_init, la_prefill, la_prefill_workspace_size, la_decode_step,
     la_device_status, la_status_string, la_prefill_path, la_resolve_chunk,
+    la_selftest_wait_timeout,
 )

@@ -58,6 +58,8 @@ def load_library():
         lib.la_prefill_workspace_size.restype = sz
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.la_device_status.argtypes = [vp]
+        lib.la_selftest_wait_timeout.argtypes = [ctypes.c_double, vp]
+        lib.la_selftest_wait_timeout.restype = ctypes.c_int
         lib.la_prefill_path.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
         lib.la_prefill_path.restype = ctypes.c_char_p
         lib.la_resolve_chunk.argtypes = [i32, i32, i32, i32]
@@ -168,6 +170,12 @@ def la_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.T
 def la_device_status(stream=None) -> int:
     """Synchronise the stream; return the device status code (LA_OK if clean)."""
     return int(load_library().la_device_status(_stream(stream)))
+
+
+def la_selftest_wait_timeout(timeout_ms: float = 50.0, stream=None) -> None:
+    """Launch the bounded-wait diagnostic (see include/linattn.h)."""
+    _check(load_library().la_selftest_wait_timeout(float(timeout_ms), _stream(stream)),
+           "la_selftest_wait_timeout")
 
 
 def la_prefill_path(dtype: torch.dtype, dk: int, dv: int, chunk: int = 0,

@@ -140,7 +140,8 @@ SplitPlan plan_split(int64_t n_units, int64_t T, int dk, int dv, int chunk, int 
     sp.sub_len = seg_len / k;
     sp.subs_per_seg = k;
     sp.subs_per_unit = static_cast<int>((P - 1) * k);
-    sp.bytes = static_cast<size_t>(n_units) * sp.subs_per_unit * dk * dv * sizeof(float);
+    // sub-segment sums, then one start state per later segment
+    sp.bytes = static_cast<size_t>(n_units) * (sp.subs_per_unit + sp.seg_count) * dk * dv * sizeof(float);
     return sp;
 }
 
@@ -249,6 +250,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     p.subs_per_seg = 0;
     p.subs_per_unit = 0;
     p.sub_states = nullptr;
+    p.seg_states = nullptr;
     {
         const char* pf = getenv("LINATTN_PREFETCH");
         p.prefetch = pf ? atoi(pf) : 1;  // measured best on B200 (deeper prefetch thrashes)
@@ -276,8 +278,13 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
                 p.sub_len = sp.sub_len;
                 p.subs_per_seg = sp.subs_per_seg;
                 p.subs_per_unit = sp.subs_per_unit;
-                p.sub_states = static_cast<const float*>(workspace);
-                e = launch_subsegment_states(p, tk, tv, static_cast<float*>(workspace), sms, s);
+                float* sub = static_cast<float*>(workspace);
+                float* seg = sub + static_cast<size_t>(n_units) * sp.subs_per_unit * d_k * d_v;
+                p.sub_states = sub;
+                p.seg_states = seg;
+                e = launch_subsegment_states(p, tk, tv, sub, sms, s);
+                if (e != cudaSuccess) return cuda_fail(e);
+                e = launch_segment_prefix(p, seg, s);
                 if (e != cudaSuccess) return cuda_fail(e);
             }
         }
@@ -349,6 +356,33 @@ la_status la_prefill_noalloc(const void* q, const void* k, const void* v, void* 
     }
     return la_prefill(q, k, v, o, state, dtype, B, H, T, d_k, d_v, cu_seqlens, num_seqs, max_seqlen, chunk, scratch,
                       scratch ? static_cast<size_t>(LA_NOALLOC_SCRATCH_BYTES) : 0, stream);
+}
+
+}  // extern "C"
+
+namespace la {
+// One thread waits on an mbarrier that nothing arrives on, through the same
+// bounded wait as the prefill kernels; it gives up after timeout_ns.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        mbar_wait(&bar, 0, &abort_flag, timeout_ns, 0xF00);
+    }
+}
+}  // namespace la
+
+extern "C" {
+
+la_status la_selftest_wait_timeout(double timeout_ms, void* stream) {
+    if (!(timeout_ms > 0.0) || timeout_ms > 10000.0) return LA_ERR_INVALID_ARG;
+    la::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(timeout_ms * 1e6));
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LA_OK : cuda_fail(e);
 }
 
 la_status la_device_status(void* stream) {

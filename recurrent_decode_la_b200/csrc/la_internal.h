@@ -28,16 +28,18 @@ struct PrefillProblem {
     uint64_t timeout_ns;
     // Intra-sequence split (dense input only; seg_count = 1 means none).
     // Work item i is segment i % seg_count of unit i / seg_count: rows
-    // [s * seg_len, min((s + 1) * seg_len, rows_per_group)).  Segment s starts
-    // from S_0 plus the K^T V sums of the first s * subs_per_seg sub-segments
-    // (sub_len rows each) in sub_states [units][subs_per_unit][dk][dv]; only
-    // the last segment writes S_T.
+    // [s * seg_len, min((s + 1) * seg_len, rows_per_group)).  Segment s
+    // starts from seg_states[u][s] = S_0 plus the K^T V sums of the first
+    // s * subs_per_seg sub-segments (sub_len rows each, sums kept in
+    // sub_states [units][subs_per_unit][dk][dv]); only the last segment
+    // writes S_T.
     int seg_count;
     int64_t seg_len;
     int64_t sub_len;
     int subs_per_seg;
     int subs_per_unit;
     const float* sub_states;
+    const float* seg_states;  // [units][seg_count][dk][dv]
     // Chunks ahead of the shared-memory load that the producer prefetches
     // into L2 (0 = none).
     int prefetch;
@@ -61,6 +63,10 @@ cudaError_t launch_prefill_tc(const PrefillProblem& p, const CUtensorMap& tq,
 // j < subs_per_unit (tensor cores, bf16 in, fp32 out).
 cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap& tk, const CUtensorMap& tv,
                                      float* sub_states, int num_sms, cudaStream_t s);
+
+// seg_states[u][s] = S_0[u] + sum of sub_states[u][0 .. s*subs_per_seg - 1]
+// for s = 0 .. seg_count - 1 (one pass over the sub-segment sums).
+cudaError_t launch_segment_prefix(const PrefillProblem& p, float* seg_states, cudaStream_t s);
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* state,
                           int dtype, int64_t n_units, int dk, int dv, int num_sms,

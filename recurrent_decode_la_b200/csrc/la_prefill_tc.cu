@@ -595,12 +595,15 @@ __global__ void __launch_bounds__(512, 1)
             if (nch == 0) continue;
             float* st_row = p.state + un.unit * static_cast<int64_t>(D) * D +
                             static_cast<int64_t>(rowS < 0 ? 0 : rowS) * D;
-            // a segment after the first starts from S_0 plus the K^T V sums of
-            // every sub-segment before it
-            const int nsub = un.seg * p.subs_per_seg;
-            const float* sub_row = nsub > 0 ? p.sub_states + un.unit * static_cast<int64_t>(p.subs_per_unit) * D * D +
-                                                  static_cast<int64_t>(rowS < 0 ? 0 : rowS) * D
-                                            : nullptr;
+            // a segment after the first starts from its precomputed state
+            // (S_0 plus the K^T V sums of everything before it)
+            // (with a split every segment, the first included, reads its start
+            // state from the workspace: the state buffer itself is written by
+            // the last segment and is never read by another work item)
+            const float* in_row = p.seg_count > 1 ? p.seg_states +
+                                                        (un.unit * static_cast<int64_t>(p.seg_count) + un.seg) * D * D +
+                                                        static_cast<int64_t>(rowS < 0 ? 0 : rowS) * D
+                                                  : st_row;
             // ---- unit start: S_0 into TMEM (fp32) and into the bf16 operand
             if (g > 0 && !mbar_wait_warp(&bar[Cfg::B_SBEMPTY], (g - 1) & 1, abort_flag, tmo, 0x300)) {
                 ok = false;
@@ -610,18 +613,10 @@ __global__ void __launch_bounds__(512, 1)
             for (int cb = 0; cb < D / 32; ++cb) {
                 uint32_t r[32];
                 if (rowS >= 0) {
-                    const float4* src = reinterpret_cast<const float4*>(st_row + cb * 32);
+                    const float4* src = reinterpret_cast<const float4*>(in_row + cb * 32);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        float4 f = src[i];
-                        for (int j = 0; j < nsub; ++j) {
-                            const float4 d4 = reinterpret_cast<const float4*>(
-                                sub_row + static_cast<int64_t>(j) * D * D + cb * 32)[i];
-                            f.x += d4.x;
-                            f.y += d4.y;
-                            f.z += d4.z;
-                            f.w += d4.w;
-                        }
+                        const float4 f = src[i];
                         r[4 * i + 0] = __float_as_uint(f.x);
                         r[4 * i + 1] = __float_as_uint(f.y);
                         r[4 * i + 2] = __float_as_uint(f.z);
@@ -1030,6 +1025,39 @@ cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap&
     if (p.dk == 64 && p.chunk == 128) return launch_sub_impl<128, 64>(p, tk, tv, sub_states, num_sms, s);
     if (p.dk == 128 && p.chunk == 128) return launch_sub_impl<128, 128>(p, tk, tv, sub_states, num_sms, s);
     return cudaErrorInvalidValue;
+}
+
+// seg_states[u][s] = S_0[u] + sum_{j < s*k} sub_states[u][j] for every segment
+// s (s = 0 is a copy of S_0): one thread per float4 of a unit's state walks
+// the sub-segment sums once, in order.
+__global__ void segment_prefix_kernel(const float4* __restrict__ s0, const float4* __restrict__ sub,
+                                      float4* __restrict__ seg, int64_t n_units, int d4, int subs_per_seg,
+                                      int seg_count) {
+    const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+    if (i >= n_units * d4) return;
+    const int64_t u = i / d4, e = i % d4;
+    const int subs = (seg_count - 1) * subs_per_seg;
+    float4 acc = s0[u * d4 + e];
+    seg[(u * seg_count) * d4 + e] = acc;
+    for (int j = 0; j < subs; ++j) {
+        const float4 x = sub[(u * subs + j) * d4 + e];
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
+        if ((j + 1) % subs_per_seg == 0) seg[(u * seg_count + (j + 1) / subs_per_seg) * d4 + e] = acc;
+    }
+}
+
+cudaError_t launch_segment_prefix(const PrefillProblem& p, float* seg_states, cudaStream_t s) {
+    const int d4 = p.dk * p.dv / 4;
+    const int64_t n = p.n_units * d4;
+    if (n <= 0) return cudaSuccess;
+    const int threads = 256;
+    segment_prefix_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, s>>>(
+        reinterpret_cast<const float4*>(p.state), reinterpret_cast<const float4*>(p.sub_states),
+        reinterpret_cast<float4*>(seg_states), p.n_units, d4, p.subs_per_seg, p.seg_count);
+    return cudaGetLastError();
 }
 
 bool prefill_tc_supported(int D, int chunk) {

@@ -1,6 +1,7 @@
 """Host-side checks of the C ABI that need no GPU: the library loads, exports
 every entry point declared in include/linattn.h, and answers host-only
 queries (status strings, kernel choice, argument validation before launch)."""
+import ctypes
 import os
 import re
 
@@ -73,6 +74,9 @@ def test_argument_checks_before_any_launch(lib):
     assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 0, 128) > 0
     assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 64, 128) == 0   # packed: never split
     assert lib.la_prefill_workspace_size(0, 1, 32, 131072, 128, 128, 0, 128) == 0    # fp32: CUDA-core path
+    lib.la_selftest_wait_timeout.argtypes = [ctypes.c_double, ctypes.c_void_p]
+    assert lib.la_selftest_wait_timeout(0.0, None) == la.LA_ERR_INVALID_ARG
+    assert lib.la_selftest_wait_timeout(2e4, None) == la.LA_ERR_INVALID_ARG
 
 
 def test_binding_rejects_cpu_tensors():
