@@ -174,11 +174,21 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_cols_kernel(const T* __
             }
         }
     }
-    reinterpret_cast<float4*>(red + r0 * ncol)[c4] = acc;
+    // q^T S' over this CTA's rows: first across the lanes of a warp that own
+    // the same columns (shuffles), then across the 8 warps (shared memory).
+    for (int off = cols4; off < 32; off <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+    }
+    const int lane = tid & 31, wid = tid >> 5;
+    if (lane < cols4) reinterpret_cast<float4*>(red + wid * ncol)[lane] = acc;
     __syncthreads();
     for (int n = tid; n < ncol; n += kDecThreads) {
         float sum = 0.f;
-        for (int rr = 0; rr < rpp && rr < dk; ++rr) sum += red[rr * ncol + n];
+#pragma unroll
+        for (int w = 0; w < kDecThreads / 32; ++w) sum += red[w * ncol + n];
         dec_out<T>(o, u * dv + cbeg + n, sum);
     }
 }
