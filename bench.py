@@ -45,7 +45,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--chunk", type=int, default=0, help="0 = the library's default for the shape")
-    ap.add_argument("--sweep-chunks", default="64,128",
+    ap.add_argument("--sweep-chunks", default="32,64,128",
                     help="also time the prefill alone at these chunk sizes ('' = none)")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
     ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end run")
@@ -481,6 +481,133 @@ def chunk_sweep(la, torch, stream, q, k, v, o, state, wl, chunks, peaks, dev):
     return out
 
 
+def run_varlen(args, wl, world, rank, local):
+    """Packed variable-length workload: one step = prefill of every packed
+    sequence (la_prefill with cu_seqlens), the prefilled states tiled
+    decode_repeat times (la_state_init copies), then decode steps for all those
+    states.  Same timing rules and JSON keys as the dense workload."""
+    import concurrent.futures
+    import torch
+    import torch.distributed as dist
+
+    import recurrent_decode_la_b200 as la
+    from recurrent_decode_la_b200 import inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    la.load_library()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks, peak_src = load_peaks()
+    H, d, N, rep = wl.H, wl.d, wl.num_seqs, wl.decode_repeat
+    chunk = args.chunk or la.la_resolve_chunk(wl.torch_dtype, d, d, 0)
+    dsteps = wl.decode_steps if args.decode_steps < 0 else args.decode_steps
+    q_h, k_h, v_h, cu = inputs.prefill_inputs(wl)
+    Ttot = q_h.shape[2]
+    max_len = int((cu[1:] - cu[:-1]).max())
+    units, dunits, bdec = N * H, inputs.decode_units(wl), N * rep
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        toks = list(ex.map(lambda s_: inputs.decode_token(wl, s_, units=dunits), range(dsteps)))
+    q, k, v, cud = q_h.to(dev), k_h.to(dev), v_h.to(dev), cu.to(dev)
+    shape = (dsteps, bdec, H, d)
+    dq = torch.stack([t[0] for t in toks]).reshape(shape).to(dev) if dsteps else None
+    dk_ = torch.stack([t[1] for t in toks]).reshape(shape).to(dev) if dsteps else None
+    dv = torch.stack([t[2] for t in toks]).reshape(shape).to(dev) if dsteps else None
+    del toks
+    o = torch.empty_like(v)
+    od = torch.empty_like(dv) if dsteps else None
+    st_p = torch.empty(units, d, d, dtype=torch.float32, device=dev)
+    st_d = torch.empty(dunits, d, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def prefill_phase(s_):
+        la.la_state_init(st_p, None, stream=s_)
+        la.la_prefill(q, k, v, o, st_p, cu_seqlens=cud, max_seqlen=max_len, chunk=chunk, stream=s_)
+        for r in range(rep):
+            la.la_state_init(st_d[r * units:(r + 1) * units], st_p, stream=s_)
+
+    def decode_phase(s_):
+        for i in range(dsteps):
+            la.la_decode_step(dq[i], dk_[i], dv[i], od[i], st_d, stream=s_)
+
+    with torch.cuda.stream(stream):
+        prefill_phase(stream)
+        if dsteps:
+            decode_phase(stream)
+    stream.synchronize()
+    g_pre = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_pre, stream=stream):
+        prefill_phase(torch.cuda.current_stream())
+    g_dec = None
+    if dsteps:
+        g_dec = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_dec, stream=stream):
+            decode_phase(torch.cuda.current_stream())
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            g_pre.replay()
+            if g_dec is not None:
+                g_dec.replay()
+    stream.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                ev[i][0].record(stream)
+                g_pre.replay()
+                ev[i][1].record(stream)
+                if g_dec is not None:
+                    g_dec.replay()
+                ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    status = la.la_device_status(stream)
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    dec_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) if dsteps else 0.0
+    ms_total = max_over_ranks(ev[0][0].elapsed_time(ev[-1][2]), dev)
+    tokens_step = Ttot + bdec * dsteps
+    elem = 2 if wl.dtype == "bf16" else 4
+    pre_bytes = Ttot * H * 4 * d * elem + units * 2 * d * d * 4
+    dec_bytes = decode_bytes(dunits, d, d, elem)
+    pre_gbs = pre_bytes / (pre_ms * 1e-3) / 1e9
+    dec_us = 1e3 * dec_ms / max(1, dsteps)
+    dec_gbs = dec_bytes / (dec_us * 1e-6) / 1e9 if dsteps else 0.0
+    pre_share = pre_ms / (pre_ms + dec_ms) if (pre_ms + dec_ms) > 0 else 1.0
+    roof_pre = {"bound": "hbm", "kernel": "prefill_" + la.la_prefill_path(wl.torch_dtype, d, d, chunk, q, k, v, o),
+                "achieved": pre_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": pre_gbs / peaks["hbm_gbs"],
+                "traffic": None, "bytes_per_launch": pre_bytes, "share_of_step": pre_share,
+                "peak_source": f"{peak_src} hbm_gbs"}
+    roof_dec = {"bound": "hbm", "kernel": "decode_cols", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"], "traffic": None, "bytes_per_launch": dec_bytes,
+                "share_of_step": 1 - pre_share, "note": "512 MiB of decode state: cold in every step",
+                "peak_source": f"{peak_src} hbm_gbs"}
+    result = {
+        "metric": METRIC, "value": whole_job_rate(world, args.steps, tokens_step, ms_total), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs": N, "H": H, "T_total": Ttot, "max_seqlen": max_len, "d_k": d,
+                   "d_v": d, "chunk": chunk, "decode_units": dunits, "decode_steps": dsteps,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs (%.1f GB) and decode state (512 MiB) larger than L2" % (3 * q.numel() * elem / 1e9)},
+        "prefill": {"tokens_per_s": Ttot / (pre_ms * 1e-3), "ms": pre_ms, "achieved_gbs": pre_gbs,
+                    "hbm_frac": pre_gbs / peaks["hbm_gbs"]},
+        "decode": {"tokens_per_s": bdec * dsteps / (dec_ms * 1e-3) if dsteps else 0.0, "us_per_step": dec_us,
+                   "achieved_gbs": dec_gbs, "hbm_frac": dec_gbs / peaks["hbm_gbs"] if dsteps else 0.0},
+        "roofline": roof_pre if pre_share >= 0.5 else roof_dec, "roofline_prefill": roof_pre,
+        "gpu_launches": args.steps * (2 + rep + dsteps), "device_status": la.la_status_string(status),
+        "clocks": clk.summary(), "peaks_source": peak_src,
+    }
+    del g_pre, g_dec
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
 def cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_src):
     """Decode with a cold state: rotate over R state sets larger than L2 (as a
     stack of R layers would), one launch per set, timed with CUDA events."""
@@ -524,8 +651,12 @@ def cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_
 
 
 def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h, dk_h, dv_h, world):
-    """Same step through the public API with host buffers: pinned host -> device
-    copies of every input, and device -> host copies of every output, timed."""
+    """The same step through the public API with host buffers: pinned host ->
+    device copies of every input and device -> host copies of every output,
+    all inside the timed region.  Sequences are independent, so the step is
+    pipelined per sequence on three streams: the copy-in of sequence b+1 and
+    the copy-out of sequence b-1 overlap the prefill of sequence b
+    (la_prefill on that sequence's slices); the decode steps follow."""
     B, H, T, d = wl.B, wl.H, wl.T, wl.d
     pins = [x.pin_memory() for x in (q_h, k_h, v_h, dq_h, dk_h, dv_h)]
     o_h = torch.empty_like(pins[2]).pin_memory()
@@ -535,19 +666,43 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
     o = torch.empty_like(dev_bufs[2])
     od = torch.empty_like(dev_bufs[5])
     st = torch.empty(B * H, d, d, dtype=torch.float32, device=dev)
-    nb = la.la_prefill_workspace_size(wl.torch_dtype, B, H, T, d, d, 0, chunk)
+    nb = la.la_prefill_workspace_size(wl.torch_dtype, 1, H, T, d, d, 0, chunk)
     ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
     def step():
-        for h, dbuf in zip(pins, dev_bufs):
-            dbuf.copy_(h, non_blocking=True)
-        la.la_state_init(st, None, stream=stream)
-        la.la_prefill(dev_bufs[0], dev_bufs[1], dev_bufs[2], o, st, chunk=chunk, workspace=ws, stream=stream)
+        copied = [torch.cuda.Event() for _ in range(B)]
+        done = [torch.cuda.Event() for _ in range(B)]
+        with torch.cuda.stream(s_in):
+            s_in.wait_stream(stream)
+            for b in range(B):
+                for i in range(3):
+                    dev_bufs[i][b].copy_(pins[i][b], non_blocking=True)
+                copied[b].record(s_in)
+            for i in range(3, 6):
+                dev_bufs[i].copy_(pins[i], non_blocking=True)
+            dec_in = torch.cuda.Event()
+            dec_in.record(s_in)
+        for b in range(B):
+            stream.wait_event(copied[b])
+            sl = slice(b * H, (b + 1) * H)
+            la.la_state_init(st[sl], None, stream=stream)
+            la.la_prefill(dev_bufs[0][b:b + 1], dev_bufs[1][b:b + 1], dev_bufs[2][b:b + 1], o[b:b + 1], st[sl],
+                          chunk=chunk, workspace=ws, stream=stream)
+            done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[b])
+                o_h[b].copy_(o[b], non_blocking=True)
+        stream.wait_event(dec_in)
         for i in range(dsteps):
             la.la_decode_step(dev_bufs[3][i], dev_bufs[4][i], dev_bufs[5][i], od[i], st, stream=stream)
-        o_h.copy_(o, non_blocking=True)
-        od_h.copy_(od, non_blocking=True)
-        st_h.copy_(st, non_blocking=True)
+        fin = torch.cuda.Event()
+        fin.record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(fin)
+            od_h.copy_(od, non_blocking=True)
+            st_h.copy_(st, non_blocking=True)
+        stream.wait_stream(s_out)
 
     n_steps = max(1, min(args.steps, args.e2e_steps))
     with torch.cuda.stream(stream):
@@ -566,7 +721,8 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
     tokens = B * T + B * dsteps
     return {"value": world * n_steps * tokens / (ms * 1e-3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / n_steps,
-            "steps": n_steps}
+            "steps": n_steps, "pipelined": "per sequence: copy-in / prefill / copy-out on three streams",
+            "h2d_gbs": h2d / (ms / n_steps * 1e-3) / 1e9}
 
 
 def main(argv=None):
@@ -579,6 +735,8 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
+    if wl.varlen:
+        return run_varlen(args, wl, world, rank, local)
     return run_ours(args, wl, world, rank, local)
 
 
