@@ -45,7 +45,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--chunk", type=int, default=0, help="0 = the library's default for the shape")
-    ap.add_argument("--sweep-chunks", default="32,64,128",
+    ap.add_argument("--sweep-chunks", default="16,32,64,128",
                     help="also time the prefill alone at these chunk sizes ('' = none)")
     ap.add_argument("--batch", type=int, default=0, help="override B (small profiling cases)")
     ap.add_argument("--e2e-steps", type=int, default=10, help="steps of the end-to-end run")

@@ -14,7 +14,8 @@
 // One persistent CTA per SM walks units (one sequence of one head) with a
 // static stride.  Warp roles (512 threads):
 //   warp 0       TMA producer: Q/K/V chunk tiles into an NS-deep ring
-//   warp 1       MMA issuer (one thread) and TMEM owner
+//   warps 1-3    MMA issuers (one thread each: output, state, scores);
+//                warp 1 also owns the TMEM allocation
 //   warps 4-7    "mask" warpgroup: scores -> causal mask -> bf16 P
 //   warps 8-11   "state" warpgroup: S_0 in, state hop S -> bf16 operand, S_T out
 //   warps 12-15  "output" warpgroup: O TMEM -> bf16 -> smem -> TMA store
@@ -46,31 +47,44 @@ namespace la {
 template <int C, int D>
 struct TcCfg {
     static constexpr int kThreads = 512;
-    static constexpr int PANEL = C * 128;  // one 64-column panel of a chunk tile (bytes)
+    // Rows of the attention MMAs (Q K^T, Q S, P V).  tcgen05 has no M below
+    // 64, so a chunk of 16 or 32 tokens runs M = 64 tiles whose first C rows
+    // are the chunk; the other rows of the Q and P tiles are zero and their
+    // accumulator rows are never read.
+    static constexpr int MR = C < 64 ? 64 : C;
+    static constexpr int PANEL = C * 128;   // one 64-column panel of a K/V/O chunk tile (bytes)
+    static constexpr int QPANEL = MR * 128; // one panel of the Q tile (padded to MR rows)
     static constexpr int NPAN = D / 64;
     static constexpr int TILE = C * D * 2;
-    static constexpr int STAGE = 3 * TILE;  // Q, K, V of one chunk
+    static constexpr int QTILE = MR * D * 2;
+    static constexpr int STAGE = QTILE + 2 * TILE;  // Q, K, V of one chunk
+    static constexpr int STAGE_TX = 3 * TILE;       // bytes the TMA writes into a stage
     // C = 128: P stays in tensor memory (written over the fp32 scores it came
     // from, read by the P V MMA straight from TMEM) and O is staged for its
     // TMA store in the chunk's own Q tile, which is dead by then; the shared
-    // memory this frees buys a deeper Q/K/V ring.  C = 64 (M = 64 tiles) keeps
+    // memory this frees buys a deeper Q/K/V ring.  C <= 64 (M = 64 tiles) keeps
     // P and the O staging in their own shared-memory buffers.
     static constexpr bool PT = (C == 128);
-    static constexpr int NS = PT ? (D == 128 ? 2 : 4) : (D == 64 ? 6 : 3);
     static constexpr int PB = PT ? 0 : 2;                       // P buffers in smem
     static constexpr int OB = (C == 128 && D == 128) ? 1 : 2;  // O accumulators in TMEM
     static constexpr int OSB = PT ? 0 : 2;                      // O staging buffers in smem
-    static constexpr int P_BYTES = C * C * 2;
-    static constexpr int P_PANEL = C * 128;
+    static constexpr int PK = C < 64 ? 64 : C;                  // P row width (keys, padded)
+    static constexpr int P_BYTES = MR * PK * 2;
+    static constexpr int P_PANEL = MR * 128;
     static constexpr int SB_BYTES = D * D * 2;
     static constexpr int SB_PANEL = D * 128;
     static constexpr int OST_BYTES = C * D * 2;
+    static constexpr int NBAR = 48;
+    static constexpr int FIXED = PB * P_BYTES + SB_BYTES + OSB * OST_BYTES + NBAR * 8 + 16 + 1024;
+    // ring depth: C = 128 and C = 64 as tuned; smaller chunks as deep as fits (<= 8)
+    static constexpr int NS_FIT = (232448 - FIXED) / STAGE;
+    static constexpr int NS = PT ? (D == 128 ? 2 : 4)
+                                 : (C == 64 ? (D == 64 ? 6 : 3) : (NS_FIT < 8 ? NS_FIT : 8));
     static constexpr int OFF_STAGE = 0;
     static constexpr int OFF_P = OFF_STAGE + NS * STAGE;
     static constexpr int OFF_SB = OFF_P + PB * P_BYTES;
     static constexpr int OFF_OST = OFF_SB + SB_BYTES;
     static constexpr int OFF_BAR = OFF_OST + OSB * OST_BYTES;
-    static constexpr int NBAR = 48;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
     // tensor memory columns (fp32, 128 lanes)
@@ -78,9 +92,11 @@ struct TcCfg {
     static constexpr int TM_O = D;
     static constexpr int TM_A = D + OB * D;
     static constexpr int TM_COLS = 512;
-    static_assert(TM_A + 2 * C <= TM_COLS, "tensor memory budget");
+    static constexpr int A_COLS = C < 64 ? 64 : C;  // columns per score buffer (64-aligned)
+    static_assert(C % 16 == 0 && C >= 16 && C <= 128, "chunk size");
+    static_assert(TM_A + 2 * A_COLS <= TM_COLS, "tensor memory budget");
     static_assert(SMEM <= 232448, "shared memory budget");
-    static_assert(NS <= 6, "barrier slots");
+    static_assert(NS >= 2 && NS <= 8, "barrier slots");
     // mbarrier slots
     static constexpr int B_FULL = 0;       // [NS] TMA landed
     static constexpr int B_EMPTY = 8;      // [NS] MMAs of the stage done
@@ -96,7 +112,7 @@ struct TcCfg {
     static constexpr int B_OEMPTY = 30;    // [2] O read out
     static constexpr int B_OSTFULL = 32;   // [2] O staging written
     static constexpr int B_OSTFREE = 34;   // [2] O staging read by the TMA store
-    static constexpr int B_MMADONE = 36;   // [2] drain at teardown (one per issuing thread)
+    static constexpr int B_MMADONE = 36;   // [3] drain at teardown (one per issuing thread)
     static constexpr int B_ZERO = 40;      // [NS] rows past the sequence end zeroed in K, V
 };
 
@@ -179,8 +195,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(&bar[Cfg::B_SREAD], 4);
         mbar_init(&bar[Cfg::B_SBFULL], 4);
         mbar_init(&bar[Cfg::B_SBEMPTY], 1);
-        mbar_init(&bar[Cfg::B_MMADONE], 1);
-        mbar_init(&bar[Cfg::B_MMADONE + 1], 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[Cfg::B_MMADONE + i], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -193,6 +208,20 @@ __global__ void __launch_bounds__(512, 1)
     if (warp == 1) {
         tmem_alloc(tmem_base_slot, Cfg::TM_COLS);
         tmem_relinquish();
+    }
+    if constexpr (Cfg::MR > C) {
+        // Pad rows C..MR-1 of every Q panel and of the P tiles: zero once,
+        // never written again (the TMA fills rows 0..C-1 only).
+        constexpr int kPad = (Cfg::MR - C) * 128 / 16;  // 16-byte pieces per panel
+        const uint32_t sb = smem_u32(smem);
+        for (int i = threadIdx.x; i < (Cfg::NS * Cfg::NPAN + Cfg::PB) * kPad; i += blockDim.x) {
+            const int t = i / kPad, r = i % kPad;
+            const uint32_t panel = t < Cfg::NS * Cfg::NPAN
+                                       ? Cfg::OFF_STAGE + (t / Cfg::NPAN) * Cfg::STAGE + (t % Cfg::NPAN) * Cfg::QPANEL
+                                       : Cfg::OFF_P + (t - Cfg::NS * Cfg::NPAN) * Cfg::P_BYTES;
+            st_shared_v4(sb + panel + C * 128 + r * 16, 0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -209,8 +238,8 @@ __global__ void __launch_bounds__(512, 1)
 
     const uint32_t sbase = smem_u32(smem);
     auto stage_q = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE; };
-    auto stage_k = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + Cfg::TILE; };
-    auto stage_v = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + 2 * Cfg::TILE; };
+    auto stage_k = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + Cfg::QTILE; };
+    auto stage_v = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + Cfg::QTILE + Cfg::TILE; };
     const uint32_t p_base = sbase + Cfg::OFF_P;
     const uint32_t sb_base = sbase + Cfg::OFF_SB;
     const uint32_t ost_base = sbase + Cfg::OFF_OST;
@@ -234,11 +263,11 @@ __global__ void __launch_bounds__(512, 1)
                             break;
                         }
                     }
-                    mbar_arrive_expect_tx(&bar[Cfg::B_FULL + s], Cfg::STAGE);
+                    mbar_arrive_expect_tx(&bar[Cfg::B_FULL + s], Cfg::STAGE_TX);
                     const int row = un.row0 + c * C;
 #pragma unroll
                     for (int pn = 0; pn < Cfg::NPAN; ++pn) {
-                        tma_load_3d(reinterpret_cast<void*>(smem + (stage_q(s) - sbase) + pn * Cfg::PANEL),
+                        tma_load_3d(reinterpret_cast<void*>(smem + (stage_q(s) - sbase) + pn * Cfg::QPANEL),
                                     &tmQ, &bar[Cfg::B_FULL + s], pn * 64, row, un.group);
                         tma_load_3d(reinterpret_cast<void*>(smem + (stage_k(s) - sbase) + pn * Cfg::PANEL),
                                     &tmK, &bar[Cfg::B_FULL + s], pn * 64, row, un.group);
@@ -267,22 +296,20 @@ __global__ void __launch_bounds__(512, 1)
                         mbar_wait_drain(&bar[Cfg::B_FULL + s], (last_g[s] / Cfg::NS) & 1, tmo);
             }
         }
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp >= 1 && warp <= 3) {
         // ----------------------------------------------------- MMA issuers
-        // Two threads issue tcgen05 MMAs; an issuing thread blocks while the
-        // tensor pipe is busy, so splitting the work keeps one stream going
-        // while the other waits on a warpgroup:
-        //   warp 1 (chunk attention): A = Q K^T, O = Q S_prev, O += P V.  The
-        //     scores of chunk g+1 are issued between the two O MMAs of chunk g
-        //     when its tiles have already landed (never blocking on a load).
+        // Three threads issue tcgen05 MMAs.  An issuing thread blocks while the
+        // tensor pipe is busy, so each stream waits only on its own inputs:
+        //   warp 3 (scores): A = Q K^T as soon as the chunk's tiles have landed
+        //     and its score buffer is free.
+        //   warp 1 (output): O = Q S_prev once the bf16 state operand is
+        //     written, then O += P V once the mask warpgroup has written P.
         //   warp 2 (state carry): rows past a sequence end are zeroed in K and
         //     V, then S += K^T V as soon as the previous state has been read.
-        constexpr uint32_t kIdQK = idesc_bf16_f32(C, C, false, false);
+        constexpr uint32_t kIdQK = idesc_bf16_f32(Cfg::MR, C, false, false);
         constexpr uint32_t kIdKV = idesc_bf16_f32(D, D, true, true);
-        constexpr uint32_t kIdQS = idesc_bf16_f32(C, D, false, true);
-        constexpr uint32_t kIdPV = idesc_bf16_f32(C, D, false, true);
-        constexpr bool kLookahead = Cfg::NS >= 2;
-        const bool attn = (warp == 1);
+        constexpr uint32_t kIdQS = idesc_bf16_f32(Cfg::MR, D, false, true);
+        constexpr uint32_t kIdPV = idesc_bf16_f32(Cfg::MR, D, false, true);
         bool ok = true;
         bool issued_any = false;
         // (unit, chunk) walk
@@ -325,7 +352,7 @@ __global__ void __launch_bounds__(512, 1)
             k.valid = false;
         };
 
-        if (!attn) {
+        if (warp == 2) {
             // ------------------------------------------------ state stream
             const uint32_t tm_S = tmem + Cfg::TM_S;
             Cursor k;
@@ -372,51 +399,59 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
             }
-        } else {
-            // -------------------------------------------- attention stream
-            auto issue_scores = [&](const Cursor& k) -> bool {
-                const int s = static_cast<int>(k.g % Cfg::NS);
-                if (!mbar_wait_warp(&bar[Cfg::B_FULL + s], (k.g / Cfg::NS) & 1, abort_flag, tmo, 0x208 + s))
-                    return false;
-                if (lane == 0) LA_TRACE(2, k.g);
+        } else if (warp == 3) {
+            // ----------------------------------------------- scores stream
+            Cursor k;
+            for (first(k); ok && k.valid; advance(k)) {
+                const int64_t g = k.g;
+                const int s = static_cast<int>(g % Cfg::NS);
+                const int b = static_cast<int>(g & 1);
+                if (!mbar_wait_warp(&bar[Cfg::B_FULL + s], (g / Cfg::NS) & 1, abort_flag, tmo, 0x208 + s)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) LA_TRACE(2, g);
                 int okw = 1;
                 if (lane == 0) {
-                    const int b = static_cast<int>(k.g & 1);
-                    if (k.g >= 2 && !mbar_wait(&bar[Cfg::B_AEMPTY + b], ((k.g >> 1) + 1) & 1, abort_flag, tmo,
-                                               0x210 + b))
+                    // buffer b was last used by chunk g-2: its scores have been
+                    // read, and (P in TMEM) its P V has completed
+                    if (g >= 2 &&
+                        !mbar_wait(&bar[Cfg::B_AEMPTY + b], ((g >> 1) + 1) & 1, abort_flag, tmo, 0x210 + b))
+                        okw = 0;
+                    if (Cfg::PT && okw && g >= 2 &&
+                        !mbar_wait(&bar[Cfg::B_PEMPTY + b], ((g >> 1) + 1) & 1, abort_flag, tmo, 0x218 + b))
                         okw = 0;
                     if (okw) {
                         tc_fence_after();
-                        const uint32_t tm_A = tmem + Cfg::TM_A + b * C;
+                        const uint32_t tm_A = tmem + Cfg::TM_A + b * Cfg::A_COLS;
                         const uint32_t qb = stage_q(s), kb = stage_k(s);
 #pragma unroll
                         for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t off = (ks >> 2) * Cfg::PANEL + (ks & 3) * 32;
-                            mma_bf16_ss(tm_A, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                            const uint32_t qoff = (ks >> 2) * Cfg::QPANEL + (ks & 3) * 32;
+                            const uint32_t koff = (ks >> 2) * Cfg::PANEL + (ks & 3) * 32;
+                            mma_bf16_ss(tm_A, sdesc_sw128(qb + qoff, 16, 1024), sdesc_sw128(kb + koff, 16, 1024),
                                         kIdQK, ks > 0);
                         }
                         mma_commit(&bar[Cfg::B_AFULL + b]);
-                        LA_TRACE(3, k.g);
+                        issued_any = true;
+                        LA_TRACE(3, g);
                     }
                 }
-                return __shfl_sync(0xffffffffu, okw, 0) != 0;
-            };
-
-            Cursor cur, nxt;
-            first(cur);
-            nxt = cur;
-            if (cur.valid) {
-                ok = issue_scores(cur);
-                issued_any = true;
-                advance(nxt);
+                ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
             }
-            while (ok && cur.valid) {
-                const int64_t g = cur.g;
+        } else {
+            // ----------------------------------------------- output stream
+            Cursor k;
+            for (first(k); ok && k.valid; advance(k)) {
+                const int64_t g = k.g;
                 const int s = static_cast<int>(g % Cfg::NS);
                 const int b = static_cast<int>(g & 1);
                 const int ob = static_cast<int>(g % Cfg::OB);
                 const uint32_t tm_O = tmem + Cfg::TM_O + ob * D;
-                bool next_scored = false;
+                if (!mbar_wait_warp(&bar[Cfg::B_FULL + s], (g / Cfg::NS) & 1, abort_flag, tmo, 0x228 + s)) {
+                    ok = false;
+                    break;
+                }
                 int okw = 1;
                 if (lane == 0) {
                     // O = Q S_prev
@@ -430,32 +465,16 @@ __global__ void __launch_bounds__(512, 1)
                         const uint32_t qb = stage_q(s);
 #pragma unroll
                         for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t off = (ks >> 2) * Cfg::PANEL + (ks & 3) * 32;
+                            const uint32_t off = (ks >> 2) * Cfg::QPANEL + (ks & 3) * 32;
                             mma_bf16_ss(tm_O, sdesc_sw128(qb + off, 16, 1024),
                                         sdesc_sw128(sb_base + ks * 2048, Cfg::SB_PANEL, 1024), kIdQS, ks > 0);
                         }
                         mma_commit(&bar[Cfg::B_SBEMPTY]);
+                        issued_any = true;
                     }
-                }
-                okw = __shfl_sync(0xffffffffu, okw, 0);
-                if (!okw) break;
-                // Look ahead without blocking: if the next chunk's tiles have
-                // landed, issue its scores now so the mask warpgroup can start
-                // on them while this chunk's P V runs.
-                if (kLookahead && nxt.valid) {
-                    int ready = 0;
-                    if (lane == 0)
-                        ready = mbar_try_wait(&bar[Cfg::B_FULL + static_cast<int>(nxt.g % Cfg::NS)],
-                                              (nxt.g / Cfg::NS) & 1) ? 1 : 0;
-                    if (__shfl_sync(0xffffffffu, ready, 0)) {
-                        if (!issue_scores(nxt)) break;
-                        next_scored = true;
-                    }
-                }
-                if (lane == 0) {
                     // O += P V (a partial chunk also waits for its zeroed V rows)
-                    if (!mbar_wait(&bar[Cfg::B_PFULL + b], (g >> 1) & 1, abort_flag, tmo, 0x250 + b)) okw = 0;
-                    if (okw && cur.nv < C &&
+                    if (okw && !mbar_wait(&bar[Cfg::B_PFULL + b], (g >> 1) & 1, abort_flag, tmo, 0x250 + b)) okw = 0;
+                    if (okw && k.nv < C &&
                         !mbar_wait(&bar[Cfg::B_ZERO + s], (g / Cfg::NS) & 1, abort_flag, tmo, 0x260 + s))
                         okw = 0;
                     LA_TRACE(6, g);
@@ -463,11 +482,12 @@ __global__ void __launch_bounds__(512, 1)
                         tc_fence_after();
                         const uint32_t vb = stage_v(s);
                         if constexpr (Cfg::PT) {
-                            const uint32_t tm_P = tmem + Cfg::TM_A + b * C;  // 8 columns per 16 keys
+                            const uint32_t tm_P = tmem + Cfg::TM_A + b * Cfg::A_COLS;  // 8 columns per 16 keys
 #pragma unroll
                             for (int ks = 0; ks < C / 16; ++ks)
                                 mma_bf16_ts(tm_O, tm_P + ks * 8, sdesc_sw128(vb + ks * 2048, Cfg::PANEL, 1024),
                                             kIdPV, 1);
+                            mma_commit(&bar[Cfg::B_PEMPTY + b]);
                             mma_commit(&bar[Cfg::B_OFULL + ob]);
                         } else {
                             const uint32_t pb = p_base + b * Cfg::P_BYTES;
@@ -484,27 +504,20 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, okw, 0) != 0;
-                if (!ok) break;
-                cur = nxt;
-                if (nxt.valid) {
-                    if (!next_scored) {
-                        if (!issue_scores(cur)) break;
-                    }
-                    advance(nxt);
-                }
             }
         }
         if (lane == 0 && issued_any) {
             // Drain: every MMA this thread issued has completed before TMEM is freed.
-            mma_commit(&bar[attn ? Cfg::B_MMADONE : Cfg::B_MMADONE + 1]);
-            mbar_wait_drain(&bar[attn ? Cfg::B_MMADONE : Cfg::B_MMADONE + 1], 0, tmo);
+            mma_commit(&bar[Cfg::B_MMADONE + warp - 1]);
+            mbar_wait_drain(&bar[Cfg::B_MMADONE + warp - 1], 0, tmo);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 8) {
         // ----------------------------------------------------- mask warpgroup
         const int sub = warp & 3;
         const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-        const int rowA = acc_row<C>(sub, lane);  // score / P row
+        const int rowA0 = acc_row<Cfg::MR>(sub, lane);
+        const int rowA = rowA0 < C ? rowA0 : -1;  // score / P row (-1: none, or a pad row)
         int64_t g = 0;
         bool ok = true;
         for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
@@ -524,7 +537,7 @@ __global__ void __launch_bounds__(512, 1)
                     ok = false;
                     break;
                 }
-                const uint32_t tm_A = tmem + Cfg::TM_A + b * C + lane_off;
+                const uint32_t tm_A = tmem + Cfg::TM_A + b * Cfg::A_COLS + lane_off;
                 const uint32_t pb = p_base + b * Cfg::P_BYTES;
                 if constexpr (Cfg::PT) {
                     // P (bf16 pairs) over the first C/2 columns of the scores:
@@ -548,6 +561,24 @@ __global__ void __launch_bounds__(512, 1)
                         tmem_st32(tm_A + h * 32, w);
                     }
                     tmem_wait_st();
+                } else if constexpr (C == 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tm_A, r);
+                    tmem_wait_ld();
+                    if (rowA >= 0) {
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = ch * 8 + 2 * e;
+                                const float a0 = (j <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e]) : 0.f;
+                                const float a1 = (j + 1 <= rowA) ? __uint_as_float(r[ch * 8 + 2 * e + 1]) : 0.f;
+                                w[e] = pack_bf16x2(a0, a1);
+                            }
+                            st_shared_v4(pb + sw128_off(rowA, ch), w[0], w[1], w[2], w[3]);
+                        }
+                    }
                 } else
 #pragma unroll
                 for (int cb = 0; cb < C / 32; ++cb) {
@@ -705,7 +736,8 @@ __global__ void __launch_bounds__(512, 1)
         // ---------------------------------------------------- output warpgroup
         const int sub = warp & 3;
         const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-        const int row = acc_row<C>(sub, lane);
+        const int row0 = acc_row<Cfg::MR>(sub, lane);
+        const int row = row0 < C ? row0 : -1;  // O row of this thread (-1: none, or a pad row)
         const bool elected = (warp == 12 && lane == 0);
         uint16_t* obase = static_cast<uint16_t*>(p.o);
         int64_t g = 0, f = 0;
@@ -842,7 +874,8 @@ struct KvCfg {
     static constexpr int NPAN = D / 64;
     static constexpr int TILE = C * D * 2;
     static constexpr int STAGE = 2 * TILE;  // K, V
-    static constexpr int NS = (3 * STAGE <= 200 * 1024) ? 3 : 2;
+    static constexpr int NS = C >= 64 ? ((3 * STAGE <= 200 * 1024) ? 3 : 2)
+                                      : (200 * 1024 / STAGE < 8 ? 200 * 1024 / STAGE : 8);
     static constexpr int OFF_BAR = NS * STAGE;
     static constexpr int SMEM = OFF_BAR + 32 * 8 + 16 + 1024;
     static constexpr int TM_COLS = (2 * D <= 128) ? 128 : 256;
@@ -1020,6 +1053,10 @@ static cudaError_t launch_sub_impl(const PrefillProblem& p, const CUtensorMap& t
 
 cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap& tk, const CUtensorMap& tv,
                                      float* sub_states, int num_sms, cudaStream_t s) {
+    if (p.dk == 64 && p.chunk == 16) return launch_sub_impl<16, 64>(p, tk, tv, sub_states, num_sms, s);
+    if (p.dk == 128 && p.chunk == 16) return launch_sub_impl<16, 128>(p, tk, tv, sub_states, num_sms, s);
+    if (p.dk == 64 && p.chunk == 32) return launch_sub_impl<32, 64>(p, tk, tv, sub_states, num_sms, s);
+    if (p.dk == 128 && p.chunk == 32) return launch_sub_impl<32, 128>(p, tk, tv, sub_states, num_sms, s);
     if (p.dk == 64 && p.chunk == 64) return launch_sub_impl<64, 64>(p, tk, tv, sub_states, num_sms, s);
     if (p.dk == 128 && p.chunk == 64) return launch_sub_impl<64, 128>(p, tk, tv, sub_states, num_sms, s);
     if (p.dk == 64 && p.chunk == 128) return launch_sub_impl<128, 64>(p, tk, tv, sub_states, num_sms, s);
@@ -1061,7 +1098,7 @@ cudaError_t launch_segment_prefix(const PrefillProblem& p, float* seg_states, cu
 }
 
 bool prefill_tc_supported(int D, int chunk) {
-    return (D == 64 || D == 128) && (chunk == 64 || chunk == 128);
+    return (D == 64 || D == 128) && (chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128);
 }
 
 template <int C, int D>
@@ -1091,6 +1128,10 @@ static cudaError_t launch_tc_impl(const PrefillProblem& p, const CUtensorMap& tq
 cudaError_t launch_prefill_tc(const PrefillProblem& p, const CUtensorMap& tq,
                               const CUtensorMap& tk, const CUtensorMap& tv,
                               const CUtensorMap& to, int num_sms, cudaStream_t s) {
+    if (p.dk == 64 && p.chunk == 16) return launch_tc_impl<16, 64>(p, tq, tk, tv, to, num_sms, s);
+    if (p.dk == 128 && p.chunk == 16) return launch_tc_impl<16, 128>(p, tq, tk, tv, to, num_sms, s);
+    if (p.dk == 64 && p.chunk == 32) return launch_tc_impl<32, 64>(p, tq, tk, tv, to, num_sms, s);
+    if (p.dk == 128 && p.chunk == 32) return launch_tc_impl<32, 128>(p, tq, tk, tv, to, num_sms, s);
     if (p.dk == 64 && p.chunk == 64) return launch_tc_impl<64, 64>(p, tq, tk, tv, to, num_sms, s);
     if (p.dk == 128 && p.chunk == 64) return launch_tc_impl<64, 128>(p, tq, tk, tv, to, num_sms, s);
     if (p.dk == 64 && p.chunk == 128) return launch_tc_impl<128, 64>(p, tq, tk, tv, to, num_sms, s);

@@ -88,7 +88,8 @@ def test_tiny_f32_prefill_and_decode():
 
 # ------------------------------------- tensor-core path, several tiles ----
 
-@pytest.mark.parametrize("d,chunk", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("d,chunk", [(64, 16), (128, 16), (64, 32), (128, 32),
+                                     (64, 64), (128, 64), (64, 128), (128, 128)])
 @pytest.mark.parametrize("T", [1, 63, 64, 333])
 def test_tc_prefill_random_state(d, chunk, T):
     assert la.la_prefill_path(torch.bfloat16, d, d, chunk) == "tc"
@@ -102,7 +103,8 @@ def test_tc_prefill_random_state(d, chunk, T):
 
 
 @pytest.mark.parametrize("B,H,T,d,chunk", [(1, 4, 4096, 128, 128), (1, 2, 2000, 128, 64),
-                                           (2, 3, 1111, 64, 128), (1, 1, 8192, 64, 64)])
+                                           (2, 3, 1111, 64, 128), (1, 1, 8192, 64, 64),
+                                           (1, 2, 1500, 128, 32), (1, 3, 777, 64, 16)])
 def test_intra_sequence_split(B, H, T, d, chunk):
     """Few units: each sequence is split into segments that start from S_0 plus
     the K^T V sums of the earlier sub-segments.  Same result as no split."""
@@ -120,17 +122,15 @@ def test_intra_sequence_split(B, H, T, d, chunk):
 
 
 def test_tc_vs_simt_same_inputs():
-    """Two kernels, two chunk sizes, one result (chunking never changes it)."""
+    """Two kernels, six chunk sizes, one result (chunking never changes it)."""
     q, k, v = inputs.random_qkv(3, 1, 4, 200, 64, 64, dtype=torch.bfloat16)
     O_ref, S_ref = ora.recurrent(q, k, v)
-    res = {}
-    for chunk in (16, 32, 64, 128):
+    paths = {8: "simt", 16: "tc", 32: "tc", 48: "simt", 64: "tc", 128: "tc"}
+    for chunk, path in paths.items():
+        assert la.la_prefill_path(torch.bfloat16, 64, 64, chunk) == path, chunk
         o, S = gpu_prefill(q, k, v, chunk=chunk)
-        res[chunk] = (o, S)
         assert nerr(o, O_ref) <= BF16_TOL, chunk
         assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL, chunk
-    assert la.la_prefill_path(torch.bfloat16, 64, 64, 16) == "simt"
-    assert la.la_prefill_path(torch.bfloat16, 64, 64, 64) == "tc"
 
 
 def test_misaligned_bf16_runs_simt_and_matches():
@@ -180,7 +180,7 @@ def test_varlen_small_with_empty_sequences():
     q, k, v = inputs.random_qkv(9, 1, H, int(cu[-1]), d, d, dtype=torch.bfloat16)
     S0 = torch.from_numpy(np.random.default_rng(0).standard_normal((len(lens), H, d, d)).astype(np.float32)) * 0.05
     O_ref, S_ref = ora.recurrent(q, k, v, S0, cu_seqlens=cu.numpy())
-    for chunk in (64, 128):
+    for chunk in (16, 32, 64, 128):
         o, S = gpu_prefill(q, k, v, S0=S0, cu=cu, chunk=chunk, max_seqlen=max(lens))
         assert nerr(o, O_ref) <= BF16_TOL
         assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
@@ -235,7 +235,7 @@ def test_workload_b4h8_t2048_d64_full():
     assert e_o <= BF16_TOL and e_s <= BF16_TOL
 
 
-@pytest.mark.parametrize("chunk", [64, 128])
+@pytest.mark.parametrize("chunk", [32, 64, 128])
 def test_workload_b8h16_t8192_d128_sampled(chunk):
     wl = WL["b8h16_t8192_d128_knorm"]
     q, k, v, _ = inputs.prefill_inputs(wl)

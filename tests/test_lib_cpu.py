@@ -43,6 +43,9 @@ def test_kernel_choice():
     assert la.la_prefill_path(torch.bfloat16, 128, 128, 64) == "tc"
     assert la.la_prefill_path(torch.bfloat16, 64, 64, 128) == "tc"
     assert la.la_prefill_path(torch.bfloat16, 128, 128, 128) == "tc"
+    assert la.la_prefill_path(torch.bfloat16, 128, 128, 32) == "tc"
+    assert la.la_prefill_path(torch.bfloat16, 64, 64, 16) == "tc"
+    assert la.la_prefill_path(torch.bfloat16, 128, 128, 48) == "simt"
     assert la.la_prefill_path(torch.bfloat16, 96, 96, 64) == "simt"
     assert la.la_prefill_path(torch.float32, 128, 128, 64) == "simt"
     assert la.la_prefill_path(torch.float32, 2, 2, 4) == "simt"
