@@ -520,10 +520,14 @@ def run_varlen(args, wl, world, rank, local):
     st_p = torch.empty(units, d, d, dtype=torch.float32, device=dev)
     st_d = torch.empty(dunits, d, d, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    # workspace for the longest-first order of the packed sequences
+    ws_bytes = la.la_prefill_workspace_size(wl.torch_dtype, 1, H, Ttot, d, d, N, chunk)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    ordered = ws_bytes > 0 and units > torch.cuda.get_device_properties(dev).multi_processor_count
 
     def prefill_phase(s_):
         la.la_state_init(st_p, None, stream=s_)
-        la.la_prefill(q, k, v, o, st_p, cu_seqlens=cud, max_seqlen=max_len, chunk=chunk, stream=s_)
+        la.la_prefill(q, k, v, o, st_p, cu_seqlens=cud, max_seqlen=max_len, chunk=chunk, workspace=ws, stream=s_)
         for r in range(rep):
             la.la_state_init(st_d[r * units:(r + 1) * units], st_p, stream=s_)
 
@@ -590,6 +594,7 @@ def run_varlen(args, wl, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": {"workload": wl.name, "num_seqs": N, "H": H, "T_total": Ttot, "max_seqlen": max_len, "d_k": d,
                    "d_v": d, "chunk": chunk, "decode_units": dunits, "decode_steps": dsteps,
+                   "workspace_bytes": ws_bytes, "schedule": "longest first" if ordered else "in order",
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs (%.1f GB) and decode state (512 MiB) larger than L2" % (3 * q.numel() * elem / 1e9)},
         "prefill": {"tokens_per_s": Ttot / (pre_ms * 1e-3), "ms": pre_ms, "achieved_gbs": pre_gbs,
@@ -597,7 +602,8 @@ def run_varlen(args, wl, world, rank, local):
         "decode": {"tokens_per_s": bdec * dsteps / (dec_ms * 1e-3) if dsteps else 0.0, "us_per_step": dec_us,
                    "achieved_gbs": dec_gbs, "hbm_frac": dec_gbs / peaks["hbm_gbs"] if dsteps else 0.0},
         "roofline": roof_pre if pre_share >= 0.5 else roof_dec, "roofline_prefill": roof_pre,
-        "gpu_launches": args.steps * (2 + rep + dsteps), "device_status": la.la_status_string(status),
+        "gpu_launches": args.steps * (2 + rep + dsteps + (1 if ordered else 0)),
+        "device_status": la.la_status_string(status),
         "clocks": clk.summary(), "peaks_source": peak_src,
     }
     del g_pre, g_dec

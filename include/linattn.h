@@ -78,23 +78,29 @@ la_status la_state_init(float* state, const float* src, int64_t n_units,
  *     (host value); ignored for dense input.
  *   chunk: C, the number of tokens per chunk; 0 picks the default for the
  *     shape (LINATTN_CHUNK in the environment overrides the default).
- *   workspace / workspace_bytes: device scratch of at least
- *     la_prefill_workspace_size() bytes (may be NULL when that is 0).
+ *   workspace / workspace_bytes: device scratch of la_prefill_workspace_size()
+ *     bytes, 16-byte aligned, owned by the caller and free for the library
+ *     until the call's work on `stream` has finished.  It buys speed only:
+ *     with less (or NULL) the call skips what the scratch is for (the split
+ *     of few long sequences into segments; the dynamic, longest-first walk
+ *     of packed sequences) and gives the same results.
  * Kernels: bf16 with d_k == d_v in {64, 128}, 16-byte aligned q/k/v/o and
- * chunk in {64, 128} run on the tensor cores (TMA + tcgen05, fp32
+ * chunk in {16, 32, 64, 128} run on the tensor cores (TMA + tcgen05, fp32
  * accumulation, fp32 state on chip); everything else with d_k, d_v <= 128
  * runs the fp32 CUDA-core kernel.  Errors: LA_ERR_INVALID_ARG (NULL tensor
- * with T > 0, B/H/T/d negative, B != 1 with cu_seqlens, workspace too
- * small), LA_ERR_UNSUPPORTED (d_k or d_v above 128, a chunk the kernels
- * cannot stage in shared memory). */
+ * with T > 0, B/H/T/d negative, B != 1 with cu_seqlens), LA_ERR_UNSUPPORTED
+ * (d_k or d_v above 128, a chunk the kernels cannot stage in shared
+ * memory). */
 la_status la_prefill(const void* q, const void* k, const void* v, void* o,
                      float* state, la_dtype dtype, int B, int H, int64_t T,
                      int d_k, int d_v, const int32_t* cu_seqlens, int num_seqs,
                      int64_t max_seqlen, int chunk, void* workspace,
                      size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace la_prefill needs for these arguments (0 when it
- * needs none). */
+/* Bytes of device workspace la_prefill can use for these arguments (0 when
+ * it uses none): segment states of the intra-sequence split (dense input),
+ * or, for packed input, a work counter (256 bytes) followed by one int32 per
+ * sequence (2 to 4096 sequences) for the longest-first order. */
 size_t la_prefill_workspace_size(la_dtype dtype, int B, int H, int64_t T,
                                  int d_k, int d_v, int num_seqs, int chunk);
 

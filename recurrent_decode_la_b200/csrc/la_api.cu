@@ -145,6 +145,15 @@ SplitPlan plan_split(int64_t n_units, int64_t T, int dk, int dv, int chunk, int 
     return sp;
 }
 
+// Packed input: a 256-byte slot for the work counter, then the length order
+// (one int32 per sequence, 2 to kMaxOrderedSeqs sequences).
+size_t packed_ws_bytes(int num_seqs) {
+    const size_t order = (num_seqs >= 2 && num_seqs <= kMaxOrderedSeqs)
+                             ? (static_cast<size_t>(num_seqs) * 4 + 255) / 256 * 256
+                             : 0;
+    return 256 + order;
+}
+
 enum Path { kTc, kSimt, kUnsupported };
 
 Path choose_path(la_dtype dtype, int dk, int dv, int chunk, const void* q, const void* k, const void* v,
@@ -201,11 +210,12 @@ la_status la_state_init(float* state, const float* src, int64_t n_units, int d_k
 
 size_t la_prefill_workspace_size(la_dtype dtype, int B, int H, int64_t T, int d_k, int d_v, int num_seqs,
                                  int chunk) {
-    // Only dense bf16 input on the tensor-core path is split; packed input
-    // (num_seqs > 0) never is.
-    if (num_seqs > 0 || B <= 0 || H <= 0 || T <= 0) return 0;
+    // Tensor-core path only: dense input may be split (segment states);
+    // packed input is walked dynamically (work counter + length order).
+    if (B <= 0 || H <= 0 || T <= 0) return 0;
     const int c = la_resolve_chunk(dtype, d_k, d_v, chunk);
     if (!(dtype == LA_BF16 && d_k == d_v && prefill_tc_supported(d_k, c))) return 0;
+    if (num_seqs > 0) return packed_ws_bytes(num_seqs);
     return plan_split(static_cast<int64_t>(B) * H, T, d_k, d_v, c, current_sm_count()).bytes;
 }
 
@@ -251,6 +261,8 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     p.subs_per_unit = 0;
     p.sub_states = nullptr;
     p.seg_states = nullptr;
+    p.work_counter = nullptr;
+    p.order = nullptr;
     {
         const char* pf = getenv("LINATTN_PREFETCH");
         p.prefetch = pf ? atoi(pf) : 1;  // measured best on B200 (deeper prefetch thrashes)
@@ -267,6 +279,21 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
             !encode_bf16_map(&tv, v, d_v, T, groups, c) || !encode_bf16_map(&to, o, d_v, T, groups, c)) {
             snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
             return LA_ERR_CUDA;
+        }
+        // Packed sequences, more units than SMs: the persistent CTAs claim
+        // units from a counter (so lengths that differ, and SMs that run at
+        // different speeds, even out), longest sequences first.
+        if (cu_seqlens && n_units > sms && workspace && workspace_bytes >= 256 && aligned16(workspace)) {
+            unsigned int* counter = static_cast<unsigned int*>(workspace);
+            e = cudaMemsetAsync(counter, 0, sizeof(unsigned int), s);
+            if (e != cudaSuccess) return cuda_fail(e);
+            p.work_counter = counter;
+            if (num_seqs >= 2 && num_seqs <= kMaxOrderedSeqs && workspace_bytes >= packed_ws_bytes(num_seqs)) {
+                int32_t* order = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + 256);
+                e = launch_length_order(cu_seqlens, num_seqs, T, order, s);
+                if (e != cudaSuccess) return cuda_fail(e);
+                p.order = order;
+            }
         }
         // Few long sequences: split each one so that every SM gets work, when
         // the caller provided the workspace la_prefill_workspace_size asks for.

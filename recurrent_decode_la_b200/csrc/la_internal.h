@@ -40,6 +40,14 @@ struct PrefillProblem {
     int subs_per_unit;
     const float* sub_states;
     const float* seg_states;  // [units][seg_count][dk][dv]
+    // Dynamic walk (tensor-core prefill): a zeroed counter from which the
+    // persistent CTAs claim work items in turn (nullptr: CTA b takes items
+    // b, b + G, b + 2G, ...).  Packed input under the dynamic walk may also
+    // give `order`, the sequences by decreasing length: item i is then head
+    // i % H of the sequence order[i / H], so that the longest are claimed
+    // first.
+    unsigned int* work_counter;
+    const int32_t* order;
     // Chunks ahead of the shared-memory load that the producer prefetches
     // into L2 (0 = none).
     int prefetch;
@@ -52,7 +60,7 @@ struct PrefillProblem {
 cudaError_t launch_prefill_simt(const PrefillProblem& p, int num_sms, cudaStream_t s);
 size_t prefill_simt_smem_bytes(int dk, int dv, int chunk);
 
-// Tensor-core prefill (bf16, d_k == d_v == D in {64,128}, chunk in {64,128}).
+// Tensor-core prefill (bf16, d_k == d_v == D in {64,128}, chunk in {16,32,64,128}).
 bool prefill_tc_supported(int D, int chunk);
 cudaError_t launch_prefill_tc(const PrefillProblem& p, const CUtensorMap& tq,
                               const CUtensorMap& tk, const CUtensorMap& tv,
@@ -67,6 +75,12 @@ cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap&
 // seg_states[u][s] = S_0[u] + sum of sub_states[u][0 .. s*subs_per_seg - 1]
 // for s = 0 .. seg_count - 1 (one pass over the sub-segment sums).
 cudaError_t launch_segment_prefix(const PrefillProblem& p, float* seg_states, cudaStream_t s);
+
+// order[r] = the sequence of rank r when sequences are sorted by decreasing
+// length (ties: lower index first), for num_seqs <= kMaxOrderedSeqs.
+constexpr int kMaxOrderedSeqs = 4096;
+cudaError_t launch_length_order(const int32_t* cu, int num_seqs, int64_t total_rows, int32_t* order,
+                                cudaStream_t s);
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* state,
                           int dtype, int64_t n_units, int dk, int dv, int num_sms,

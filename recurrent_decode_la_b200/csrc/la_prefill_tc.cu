@@ -74,7 +74,8 @@ struct TcCfg {
     static constexpr int SB_BYTES = D * D * 2;
     static constexpr int SB_PANEL = D * 128;
     static constexpr int OST_BYTES = C * D * 2;
-    static constexpr int NBAR = 48;
+    static constexpr int NBAR = 80;
+    static constexpr int kRing = 16;  // work-item ring (dynamic walk)
     static constexpr int FIXED = PB * P_BYTES + SB_BYTES + OSB * OST_BYTES + NBAR * 8 + 16 + 1024;
     // ring depth: C = 128 and C = 64 as tuned; smaller chunks as deep as fits (<= 8)
     static constexpr int NS_FIT = (232448 - FIXED) / STAGE;
@@ -86,7 +87,8 @@ struct TcCfg {
     static constexpr int OFF_OST = OFF_SB + SB_BYTES;
     static constexpr int OFF_BAR = OFF_OST + OSB * OST_BYTES;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KB
+    static constexpr int OFF_RING = OFF_MISC + 16;
+    static constexpr int SMEM = OFF_RING + kRing * 8 + 1024;  // + slack to align the base to 1 KB
     // tensor memory columns (fp32, 128 lanes)
     static constexpr int TM_S = 0;
     static constexpr int TM_O = D;
@@ -114,6 +116,9 @@ struct TcCfg {
     static constexpr int B_OSTFREE = 34;   // [2] O staging read by the TMA store
     static constexpr int B_MMADONE = 36;   // [3] drain at teardown (one per issuing thread)
     static constexpr int B_ZERO = 40;      // [NS] rows past the sequence end zeroed in K, V
+    static constexpr int B_UFULL = 48;     // [kRing] work item published (dynamic walk)
+    static constexpr int B_UEMPTY = 64;    // [kRing] work item taken by every consumer warp
+    static constexpr int kTakers = 15;     // warps 1..15 take every item
 };
 
 struct Unit {
@@ -137,12 +142,15 @@ __device__ __forceinline__ Unit get_unit(const PrefillProblem& p, int64_t i) {
         return {static_cast<int>(u), static_cast<int>(r0), static_cast<int>(r1 - r0), u, seg,
                 seg == p.seg_count - 1};
     }
-    const int n = static_cast<int>(i / p.H);
+    // item i: head i % H of the sequence of rank i / H (in the length order
+    // when there is one)
+    const int n = p.order != nullptr ? p.order[i / p.H] : static_cast<int>(i / p.H);
     const int h = static_cast<int>(i % p.H);
     const int a = p.cu[n];
     const int b = p.cu[n + 1];
-    if (a < 0 || b < a || static_cast<int64_t>(b) > p.rows_per_group) return {h, 0, 0, i, 0, true};
-    return {h, a, b - a, i, 0, true};
+    const int64_t unit = static_cast<int64_t>(n) * p.H + h;
+    if (a < 0 || b < a || static_cast<int64_t>(b) > p.rows_per_group) return {h, 0, 0, unit, 0, true};
+    return {h, a, b - a, unit, 0, true};
 }
 
 // Accumulator row held by lane `lane` of a warp reading its TMEM
@@ -195,6 +203,10 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(&bar[Cfg::B_SREAD], 4);
         mbar_init(&bar[Cfg::B_SBFULL], 4);
         mbar_init(&bar[Cfg::B_SBEMPTY], 1);
+        for (int r = 0; r < Cfg::kRing; ++r) {
+            mbar_init(&bar[Cfg::B_UFULL + r], 1);
+            mbar_init(&bar[Cfg::B_UEMPTY + r], Cfg::kTakers);
+        }
         for (int i = 0; i < 3; ++i) mbar_init(&bar[Cfg::B_MMADONE + i], 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -240,6 +252,40 @@ __global__ void __launch_bounds__(512, 1)
     auto stage_q = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE; };
     auto stage_k = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + Cfg::QTILE; };
     auto stage_v = [&](int s) { return sbase + Cfg::OFF_STAGE + s * Cfg::STAGE + Cfg::QTILE + Cfg::TILE; };
+    // ---- work walk.  Static: item blockIdx.x + k * gridDim.x.  Dynamic (a
+    // work counter given): the producer claims items from the global counter
+    // and publishes them, in order, in a ring of kRing slots; warps 1..15 take
+    // every item from the ring.  Either way the k-th item of the walk is the
+    // same for every role; -1 ends the walk, -2 means a wait gave up.
+    const int64_t n_items = p.n_units * p.seg_count;
+    const bool dyn = p.work_counter != nullptr;
+    volatile int64_t* ring = reinterpret_cast<volatile int64_t*>(smem + Cfg::OFF_RING);
+    auto item_static = [&](int64_t k) -> int64_t {
+        const int64_t i = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
+        return i < n_items ? i : -1;
+    };
+    auto publish_item = [&](int64_t k) -> int64_t {  // producer thread only
+        if (!dyn) return item_static(k);
+        const int r = static_cast<int>(k % Cfg::kRing);
+        if (k >= Cfg::kRing &&
+            !mbar_wait(&bar[Cfg::B_UEMPTY + r], ((k / Cfg::kRing) + 1) & 1, abort_flag, tmo, 0x140))
+            return -2;
+        int64_t i = static_cast<int64_t>(atomicAdd(p.work_counter, 1u));
+        if (i >= n_items) i = -1;
+        ring[r] = i;
+        mbar_arrive(&bar[Cfg::B_UFULL + r]);
+        return i;
+    };
+    auto take_item = [&](int64_t k) -> int64_t {  // whole warp
+        if (!dyn) return item_static(k);
+        const int r = static_cast<int>(k % Cfg::kRing);
+        if (!mbar_wait_warp(&bar[Cfg::B_UFULL + r], (k / Cfg::kRing) & 1, abort_flag, tmo, 0x148)) return -2;
+        const int64_t i = ring[r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[Cfg::B_UEMPTY + r]);
+        return i;
+    };
+
     const uint32_t p_base = sbase + Cfg::OFF_P;
     const uint32_t sb_base = sbase + Cfg::OFF_SB;
     const uint32_t ost_base = sbase + Cfg::OFF_OST;
@@ -251,7 +297,12 @@ __global__ void __launch_bounds__(512, 1)
             int64_t last_g[Cfg::NS];
             for (int s = 0; s < Cfg::NS; ++s) last_g[s] = -1;
             bool ok = true;
-            for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
+            for (int64_t kk = 0; ok; ++kk) {
+                const int64_t u = publish_item(kk);
+                if (u < 0) {
+                    ok = (u == -1);
+                    break;
+                }
                 const Unit un = get_unit(p, u);
                 const int nch = (un.len + C - 1) / C;
                 for (int c = 0; c < nch; ++c, ++g) {
@@ -314,24 +365,36 @@ __global__ void __launch_bounds__(512, 1)
         bool issued_any = false;
         // (unit, chunk) walk
         struct Cursor {
-            int64_t u;
+            int64_t u;   // work item
+            int64_t kk;  // items taken so far
             int c, nch, nv;
             int64_t g;
             bool valid;
         };
-        auto first = [&](Cursor& k) {
-            k.g = 0;
-            k.c = 0;
-            for (k.u = blockIdx.x; k.u < p.n_units * p.seg_count; k.u += gridDim.x) {
-                const Unit un = get_unit(p, k.u);
-                k.nch = (un.len + C - 1) / C;
-                if (k.nch > 0) {
+        auto next_nonempty = [&](Cursor& k) {  // next item with at least one chunk
+            for (;;) {
+                const int64_t u = take_item(k.kk++);
+                if (u < 0) {
+                    k.valid = false;
+                    if (u == -2) ok = false;
+                    return;
+                }
+                const Unit un = get_unit(p, u);
+                const int nch = (un.len + C - 1) / C;
+                if (nch > 0) {
+                    k.u = u;
+                    k.c = 0;
+                    k.nch = nch;
                     k.nv = min(C, un.len);
                     k.valid = true;
                     return;
                 }
             }
-            k.valid = false;
+        };
+        auto first = [&](Cursor& k) {
+            k.g = 0;
+            k.kk = 0;
+            next_nonempty(k);
         };
         auto advance = [&](Cursor& k) {
             ++k.g;
@@ -340,16 +403,7 @@ __global__ void __launch_bounds__(512, 1)
                 k.nv = min(C, un.len - k.c * C);
                 return;
             }
-            k.c = 0;
-            for (k.u += gridDim.x; k.u < p.n_units * p.seg_count; k.u += gridDim.x) {
-                const Unit un = get_unit(p, k.u);
-                k.nch = (un.len + C - 1) / C;
-                if (k.nch > 0) {
-                    k.nv = min(C, un.len);
-                    return;
-                }
-            }
-            k.valid = false;
+            next_nonempty(k);
         };
 
         if (warp == 2) {
@@ -520,7 +574,12 @@ __global__ void __launch_bounds__(512, 1)
         const int rowA = rowA0 < C ? rowA0 : -1;  // score / P row (-1: none, or a pad row)
         int64_t g = 0;
         bool ok = true;
-        for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
+        for (int64_t kk = 0; ok; ++kk) {
+            const int64_t u = take_item(kk);
+            if (u < 0) {
+                ok = (u == -1);
+                break;
+            }
             const Unit un = get_unit(p, u);
             const int nch = (un.len + C - 1) / C;
             for (int c = 0; c < nch; ++c, ++g) {
@@ -620,7 +679,12 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t tm_S = tmem + Cfg::TM_S + lane_off;
         int64_t g = 0;
         bool ok = true;
-        for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
+        for (int64_t kk = 0; ok; ++kk) {
+            const int64_t u = take_item(kk);
+            if (u < 0) {
+                ok = (u == -1);
+                break;
+            }
             const Unit un = get_unit(p, u);
             const int nch = (un.len + C - 1) / C;
             if (nch == 0) continue;
@@ -742,7 +806,12 @@ __global__ void __launch_bounds__(512, 1)
         uint16_t* obase = static_cast<uint16_t*>(p.o);
         int64_t g = 0, f = 0;
         bool ok = true;
-        for (int64_t u = blockIdx.x; ok && u < p.n_units * p.seg_count; u += gridDim.x) {
+        for (int64_t kk = 0; ok; ++kk) {
+            const int64_t u = take_item(kk);
+            if (u < 0) {
+                ok = (u == -1);
+                break;
+            }
             const Unit un = get_unit(p, u);
             const int nch = (un.len + C - 1) / C;
             for (int c = 0; c < nch; ++c, ++g) {
@@ -1094,6 +1163,36 @@ cudaError_t launch_segment_prefix(const PrefillProblem& p, float* seg_states, cu
     segment_prefix_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, s>>>(
         reinterpret_cast<const float4*>(p.state), reinterpret_cast<const float4*>(p.sub_states),
         reinterpret_cast<float4*>(seg_states), p.n_units, d4, p.subs_per_seg, p.seg_count);
+    return cudaGetLastError();
+}
+
+// Rank of every sequence when sorted by decreasing length (ties: lower index
+// first): each thread counts the sequences that sort before its own, over a
+// copy of all lengths in shared memory.
+__global__ void length_order_kernel(const int32_t* __restrict__ cu, int num_seqs, int64_t total_rows,
+                                    int32_t* __restrict__ order) {
+    __shared__ int32_t len[kMaxOrderedSeqs];
+    for (int i = threadIdx.x; i < num_seqs; i += blockDim.x) {
+        const int a = cu[i], b = cu[i + 1];
+        len[i] = (a < 0 || b < a || static_cast<int64_t>(b) > total_rows) ? 0 : b - a;
+    }
+    __syncthreads();
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= num_seqs) return;
+    const int li = len[i];
+    int rank = 0;
+    for (int j = 0; j < num_seqs; ++j) {
+        const int lj = len[j];
+        rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
+    }
+    order[rank] = i;
+}
+
+cudaError_t launch_length_order(const int32_t* cu, int num_seqs, int64_t total_rows, int32_t* order,
+                                cudaStream_t s) {
+    if (num_seqs <= 0 || num_seqs > kMaxOrderedSeqs) return cudaErrorInvalidValue;
+    const int threads = 256;
+    length_order_kernel<<<(num_seqs + threads - 1) / threads, threads, 0, s>>>(cu, num_seqs, total_rows, order);
     return cudaGetLastError();
 }
 

@@ -187,6 +187,40 @@ def test_varlen_small_with_empty_sequences():
         assert torch.equal(S.reshape(S_ref.shape)[1].cpu(), S0[1])  # empty sequence untouched
 
 
+@pytest.mark.parametrize("n_seqs,H,max_len,d,chunk", [(40, 8, 700, 128, 128), (40, 8, 700, 64, 64),
+                                                     (40, 8, 700, 128, 32), (5000, 1, 24, 64, 64)])
+def test_varlen_dynamic_walk(n_seqs, H, max_len, d, chunk):
+    """More units than SMs, mixed lengths: with the workspace the persistent
+    CTAs claim packed units from a counter, longest sequences first (up to
+    4096 sequences; beyond, in order).  Every unit must still be computed
+    exactly once, with the same arithmetic: the result equals the static walk
+    bit for bit (outputs start as NaN, so a skipped unit would show) and
+    matches the oracle."""
+    lens = np.random.default_rng(d + chunk + n_seqs).integers(0, max_len, size=n_seqs)
+    lens[[3, 17]] = 0
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    T = int(cu[-1])
+    nb = la.la_prefill_workspace_size(torch.bfloat16, 1, H, T, d, d, n_seqs, chunk)
+    assert nb == 256 + (((n_seqs * 4 + 255) // 256) * 256 if n_seqs <= 4096 else 0)
+    q, k, v = inputs.random_qkv(11 + d, 1, H, T, d, d, dtype=torch.bfloat16)
+    S0 = torch.from_numpy(np.random.default_rng(1).standard_normal((n_seqs, H, d, d)).astype(np.float32)) * 0.05
+    O_ref, S_ref = ora.recurrent(q, k, v, S0, cu_seqlens=cu.numpy())
+    res = []
+    for use_ws in (True, False, True):
+        qd, kd, vd, cud = q.cuda(), k.cuda(), v.cuda(), cu.cuda()
+        o = torch.full_like(vd, float("nan"))
+        st = S0.reshape(-1, d, d).cuda()
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if use_ws else None
+        la.la_prefill(qd, kd, vd, o, st, cu_seqlens=cud, max_seqlen=int(lens.max()), chunk=chunk, workspace=ws)
+        assert la.la_device_status() == la.LA_OK
+        res.append((o, st))
+    for o, st in res[1:]:
+        assert torch.equal(res[0][0], o)
+        assert torch.equal(res[0][1], st)
+    assert nerr(res[0][0], O_ref) <= BF16_TOL
+    assert nerr(res[0][1].reshape(S_ref.shape), S_ref) <= BF16_TOL
+
+
 def test_prefill_then_decode_equals_longer_prefill():
     B, H, T, n, d = 2, 4, 150, 12, 128
     q, k, v = inputs.random_qkv(17, B, H, T + n, d, d, dtype=torch.bfloat16)

@@ -75,7 +75,12 @@ def test_argument_checks_before_any_launch(lib):
     # the intra-sequence split needs workspace only for few, long, dense units
     assert lib.la_prefill_workspace_size(1, 8, 16, 8192, 128, 128, 0, 128) == 0
     assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 0, 128) > 0
-    assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 64, 128) == 0   # packed: never split
+    # packed: never split; a work counter, then one int32 per sequence for the
+    # longest-first order (2 to 4096 sequences)
+    assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 64, 128) == 512
+    assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 100, 128) == 768
+    assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 1, 128) == 256
+    assert lib.la_prefill_workspace_size(1, 1, 32, 131072, 128, 128, 5000, 128) == 256
     assert lib.la_prefill_workspace_size(0, 1, 32, 131072, 128, 128, 0, 128) == 0    # fp32: CUDA-core path
     lib.la_selftest_wait_timeout.argtypes = [ctypes.c_double, ctypes.c_void_p]
     assert lib.la_selftest_wait_timeout(0.0, None) == la.LA_ERR_INVALID_ARG
