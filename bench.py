@@ -5,7 +5,10 @@ One step = the whole path for one batch of synthetic input: S_0 = 0, the
 chunkwise prefill of every sequence (la_prefill), then `decode_steps` decode
 tokens per sequence (la_decode_step), all through the C ABI.  Default
 workload: B=8 sequences x H=16 heads, T=8192 tokens, d_k=d_v=128, bf16
-inputs with L2-normalised keys, chunk 64, 256 decode steps.
+inputs with L2-normalised keys, 256 decode steps; the prefill runs the
+library's default chunk (128), and a chunk sweep (16, 32, 64, 128) times the
+prefill alone.  Also reported outside the timed step: decode with a cold
+state, and the few-token prefill (8 tokens per unit from a saved state).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -52,6 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--decode-steps", type=int, default=-1, help="-1 = the workload's count")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-short", action="store_true", help="skip the few-token prefill measurement")
     ap.add_argument("--no-cold-decode", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the oracle sample")
@@ -435,6 +439,9 @@ def run_ours(args, wl, world, rank, local):
 
     if not args.no_cold_decode and dsteps:
         result["decode_cold"] = cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_src)
+    if not args.no_short and wl.dtype == "bf16":
+        result["short_prefill"] = [short_prefill(la, torch, dev, stream, wl, B_, H_, 8, peaks, peak_src)
+                                   for B_, H_ in ((wl.B, wl.H), (256, 32))]
 
     if not args.no_e2e:
         result["e2e"] = e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h, dk_h, dv_h,
@@ -654,6 +661,65 @@ def cold_decode(la, torch, dev, stream, wl, units, dq, dk_, dv, od, peaks, peak_
     return {"us_per_launch": us, "units": units, "state_sets": R, "bytes_per_launch": byts,
             "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
             "tokens_per_s": wl.B / (us * 1e-6)}
+
+
+def short_prefill(la, torch, dev, stream, wl, B, H, T, peaks, peak_src):
+    """T tokens per unit from a saved state in one la_prefill call (the
+    multi-token form of decode, e.g. speculative drafts), B*H units of the
+    workload's d.  The state is cold: R state sets larger than L2 in
+    rotation, one call per set.  Timed for the few-token kernel and, for
+    comparison, for the chunked kernel the library would otherwise use."""
+    from recurrent_decode_la_b200 import inputs
+    d = wl.d
+    units = B * H
+    try:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    except Exception:
+        l2 = L2_BYTES_FALLBACK
+    per = units * d * d * 4
+    R = max(2, int(math.ceil(2.5 * l2 / per)))
+    states = torch.zeros(R, units, d, d, dtype=torch.float32, device=dev)
+    q, k, v = (x.to(dev) for x in inputs.random_qkv(4242, B, H, T, d, d, dtype=wl.torch_dtype))
+    o = torch.empty_like(v)
+    reps = max(1, 64 // R)
+    out = {"T": T, "units": units, "state_sets": R}
+    for name, short in (("short", "1"), ("chunked", "0")):
+        os.environ["LINATTN_SHORT"] = short
+        try:
+            kernel = la.la_prefill_kernel(wl.torch_dtype, T, d, d, 0, q, k, v, o, states[0])
+            with torch.cuda.stream(stream):
+                for r in range(R):
+                    la.la_prefill(q, k, v, o, states[r], stream=stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    for r in range(R):
+                        la.la_prefill(q, k, v, o, states[r], stream=torch.cuda.current_stream())
+        finally:
+            os.environ.pop("LINATTN_SHORT", None)
+        with torch.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        us = 1e3 * e0.elapsed_time(e1) / (reps * R)
+        del g
+        if name == "short":
+            elem = 2 if wl.dtype == "bf16" else 4
+            byts = units * (2 * d * d * 4 + T * 4 * d * elem)
+            gbs = byts / (us * 1e-6) / 1e9
+            out.update({"kernel": kernel, "us_per_call": us, "tokens_per_s": B * T / (us * 1e-6),
+                        "bytes_per_call": byts, "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                        "peak_source": f"{peak_src} hbm_gbs"})
+        else:
+            out["chunked"] = {"kernel": kernel, "us_per_call": us}
+    del states
+    return out
 
 
 def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h, dk_h, dv_h, world):

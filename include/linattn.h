@@ -75,7 +75,9 @@ la_status la_state_init(float* state, const float* src, int64_t n_units,
  *   cu_seqlens: NULL (dense) or num_seqs+1 int32 device offsets rising from
  *     0 to T.  They are read by the kernels, not checked on the host.
  *   max_seqlen: packed mode only, an upper bound on every sequence length
- *     (host value); ignored for dense input.
+ *     (host value; 0 = unknown); ignored for dense input.  When it is at
+ *     most 16 the few-token kernel runs, and a sequence too long for it is
+ *     left untouched and reported by la_device_status (LA_ERR_INVALID_ARG).
  *   chunk: C, the number of tokens per chunk; 0 picks the default for the
  *     shape (LINATTN_CHUNK in the environment overrides the default).
  *   workspace / workspace_bytes: device scratch of la_prefill_workspace_size()
@@ -84,8 +86,11 @@ la_status la_state_init(float* state, const float* src, int64_t n_units,
  *     with less (or NULL) the call skips what the scratch is for (the split
  *     of few long sequences into segments; the dynamic, longest-first walk
  *     of packed sequences) and gives the same results.
- * Kernels: bf16 with d_k == d_v in {64, 128}, 16-byte aligned q/k/v/o and
- * chunk in {16, 32, 64, 128} run on the tensor cores (TMA + tcgen05, fp32
+ * Kernels: at most 16 tokens per unit (T, or max_seqlen), d_v a multiple of
+ * 4 and a 16-byte aligned state run the few-token kernel: the whole input as
+ * one chunk, one pass over the state, fp32 CUDA cores.  Otherwise bf16 with
+ * d_k == d_v in {64, 128}, 16-byte aligned q/k/v/o and chunk in
+ * {16, 32, 64, 128} run on the tensor cores (TMA + tcgen05, fp32
  * accumulation, fp32 state on chip); everything else with d_k, d_v <= 128
  * runs the fp32 CUDA-core kernel.  Errors: LA_ERR_INVALID_ARG (NULL tensor
  * with T > 0, B/H/T/d negative, B != 1 with cu_seqlens), LA_ERR_UNSUPPORTED
@@ -144,8 +149,9 @@ la_status la_decode_step(const void* q, const void* k, const void* v, void* o,
 
 /* Synchronises `stream`, then reports and clears the device error word of
  * the current device: LA_ERR_TIMEOUT if a kernel gave up a bounded wait
- * (its outputs are then undefined), LA_ERR_CUDA if the synchronisation
- * failed, else LA_OK. */
+ * (its outputs are then undefined), LA_ERR_INVALID_ARG if a packed sequence
+ * was longer than the max_seqlen given to la_prefill (that unit was left
+ * untouched), LA_ERR_CUDA if the synchronisation failed, else LA_OK. */
 la_status la_device_status(void* stream);
 
 /* Diagnostic of the failure path (no counterpart on the slides): launches
@@ -157,11 +163,20 @@ la_status la_device_status(void* stream);
  * usable.  Errors: LA_ERR_INVALID_ARG for timeout_ms outside (0, 10000]. */
 la_status la_selftest_wait_timeout(double timeout_ms, void* stream);
 
-/* Which kernel la_prefill would run for these arguments: "tc" (tensor
- * cores), "simt" (fp32 CUDA cores) or "unsupported".  Host only. */
+/* Which chunked kernel la_prefill would run for these arguments: "tc"
+ * (tensor cores), "simt" (fp32 CUDA cores) or "unsupported".  Host only. */
 const char* la_prefill_path(la_dtype dtype, int d_k, int d_v, int chunk,
                             const void* q, const void* k, const void* v,
                             const void* o);
+
+/* Which kernel la_prefill runs, given also max_tokens (T for dense input,
+ * max_seqlen for packed input) and the state pointer: "short" (at most 16
+ * tokens per unit: one pass over the state, fp32 CUDA cores), "tc", "simt"
+ * or "unsupported".  Host only. */
+const char* la_prefill_kernel(la_dtype dtype, int64_t max_tokens, int d_k,
+                              int d_v, int chunk, const void* q, const void* k,
+                              const void* v, const void* o,
+                              const float* state);
 
 /* The chunk size la_prefill uses for `chunk` (resolves 0 to the default). */
 int la_resolve_chunk(la_dtype dtype, int d_k, int d_v, int chunk);

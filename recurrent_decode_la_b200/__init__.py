@@ -14,6 +14,6 @@ from .binding import (  # noqa: F401
     LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT,
     LA_F32, LA_BF16, LinAttnError, lib_path, load_library,
     la_state_init, la_prefill, la_prefill_workspace_size, la_decode_step,
-    la_device_status, la_status_string, la_prefill_path, la_resolve_chunk,
+    la_device_status, la_status_string, la_prefill_path, la_prefill_kernel, la_resolve_chunk,
     la_selftest_wait_timeout,
 )

@@ -62,6 +62,8 @@ def load_library():
         lib.la_selftest_wait_timeout.restype = ctypes.c_int
         lib.la_prefill_path.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
         lib.la_prefill_path.restype = ctypes.c_char_p
+        lib.la_prefill_kernel.argtypes = [i32, i64, i32, i32, i32, vp, vp, vp, vp, vp]
+        lib.la_prefill_kernel.restype = ctypes.c_char_p
         lib.la_resolve_chunk.argtypes = [i32, i32, i32, i32]
         lib.la_status_string.argtypes = [i32]
         lib.la_status_string.restype = ctypes.c_char_p
@@ -184,6 +186,16 @@ def la_prefill_path(dtype: torch.dtype, dk: int, dv: int, chunk: int = 0,
     if all(x is None for x in p):
         p = [256] * 4  # aligned placeholders: ask about the shape only
     return load_library().la_prefill_path(_DTYPES[dtype], dk, dv, chunk, *p).decode()
+
+
+def la_prefill_kernel(dtype: torch.dtype, max_tokens: int, dk: int, dv: int, chunk: int = 0,
+                      q=None, k=None, v=None, o=None, state=None) -> str:
+    """Which kernel la_prefill runs: "short", "tc", "simt" or "unsupported".
+    max_tokens: T (dense) or max_seqlen (packed)."""
+    p = [None if t is None else t.data_ptr() for t in (q, k, v, o, state)]
+    if all(x is None for x in p):
+        p = [256] * 5  # aligned placeholders: ask about the shape only
+    return load_library().la_prefill_kernel(_DTYPES[dtype], int(max_tokens), dk, dv, chunk, *p).decode()
 
 
 def la_resolve_chunk(dtype: torch.dtype, dk: int, dv: int, chunk: int = 0) -> int:

@@ -154,7 +154,7 @@ size_t packed_ws_bytes(int num_seqs) {
     return 256 + order;
 }
 
-enum Path { kTc, kSimt, kUnsupported };
+enum Path { kTc, kSimt, kShort, kUnsupported };
 
 Path choose_path(la_dtype dtype, int dk, int dv, int chunk, const void* q, const void* k, const void* v,
                  const void* o) {
@@ -164,6 +164,20 @@ Path choose_path(la_dtype dtype, int dk, int dv, int chunk, const void* q, const
         return kTc;
     if (prefill_simt_smem_bytes(dk, dv, chunk) <= 227 * 1024) return kSimt;
     return kUnsupported;
+}
+
+// The kernel a prefill runs: the few-token kernel when no unit has more than
+// kShortMaxTokens rows (LINATTN_SHORT=0 turns it off), else the chunked
+// tensor-core kernel, else the chunked CUDA-core kernel.
+Path choose_kernel(la_dtype dtype, int64_t max_tokens, int dk, int dv, int chunk, const void* q, const void* k,
+                   const void* v, const void* o, const void* state) {
+    if (dk < 1 || dv < 1 || dk > 128 || dv > 128 || chunk < 1) return kUnsupported;
+    const char* e = getenv("LINATTN_SHORT");
+    if (!(e && e[0] == '0') && prefill_short_supported(max_tokens, dk, dv, state)) return kShort;
+    Path path = choose_path(dtype, dk, dv, chunk, q, k, v, o);
+    // The tensor-core kernel moves state rows with 16-byte accesses.
+    if (path == kTc && !aligned16(state)) path = kSimt;
+    return path;
 }
 
 }  // namespace
@@ -200,6 +214,17 @@ const char* la_prefill_path(la_dtype dtype, int d_k, int d_v, int chunk, const v
     }
 }
 
+const char* la_prefill_kernel(la_dtype dtype, int64_t max_tokens, int d_k, int d_v, int chunk, const void* q,
+                              const void* k, const void* v, const void* o, const float* state) {
+    const int c = la_resolve_chunk(dtype, d_k, d_v, chunk);
+    switch (choose_kernel(dtype, max_tokens, d_k, d_v, c, q, k, v, o, state)) {
+        case kShort: return "short";
+        case kTc: return "tc";
+        case kSimt: return "simt";
+        default: return "unsupported";
+    }
+}
+
 la_status la_state_init(float* state, const float* src, int64_t n_units, int d_k, int d_v, void* stream) {
     if (n_units < 0 || d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
     if (n_units == 0) return LA_OK;
@@ -222,7 +247,6 @@ size_t la_prefill_workspace_size(la_dtype dtype, int B, int H, int64_t T, int d_
 la_status la_prefill(const void* q, const void* k, const void* v, void* o, float* state, la_dtype dtype, int B,
                      int H, int64_t T, int d_k, int d_v, const int32_t* cu_seqlens, int num_seqs,
                      int64_t max_seqlen, int chunk, void* workspace, size_t workspace_bytes, void* stream) {
-    (void)max_seqlen;
     if (dtype != LA_F32 && dtype != LA_BF16) return LA_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || T < 0 || d_k <= 0 || d_v <= 0) return LA_ERR_INVALID_ARG;
     if (T > 0x7fffffffLL) return LA_ERR_UNSUPPORTED;
@@ -238,11 +262,10 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     if (n_units == 0 || T == 0) return LA_OK;
     if (!q || !k || !v || !o || !state) return LA_ERR_INVALID_ARG;
     const int c = la_resolve_chunk(dtype, d_k, d_v, chunk);
-    Path path = choose_path(dtype, d_k, d_v, c, q, k, v, o);
+    // packed input: max_seqlen is the caller's bound on every sequence (0: unknown)
+    const int64_t max_tokens = cu_seqlens ? max_seqlen : T;
+    const Path path = choose_kernel(dtype, max_tokens, d_k, d_v, c, q, k, v, o, state);
     if (path == kUnsupported) return LA_ERR_UNSUPPORTED;
-    // The tensor-core kernel moves state rows with 16-byte accesses.
-    if (path == kTc && !aligned16(state)) path = kSimt;
-    if (path == kSimt && prefill_simt_smem_bytes(d_k, d_v, c) > 227 * 1024) return LA_ERR_UNSUPPORTED;
 
     PrefillProblem p;
     p.q = q; p.k = k; p.v = v; p.o = o; p.state = state;
@@ -273,6 +296,10 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int sms = current_sm_count();
     cudaError_t e;
+    if (path == kShort) {
+        e = launch_prefill_short(p, max_tokens, sms, s);
+        return e == cudaSuccess ? LA_OK : cuda_fail(e);
+    }
     if (path == kTc) {
         CUtensorMap tq, tk, tv, to;
         if (!encode_bf16_map(&tq, q, d_k, T, groups, c) || !encode_bf16_map(&tk, k, d_k, T, groups, c) ||
@@ -419,11 +446,14 @@ la_status la_device_status(void* stream) {
     e = cudaMemcpyFromSymbol(w, g_error_word, sizeof(w));
     if (e != cudaSuccess) return cuda_fail(e);
     if (w[0] != 0) {
-        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "device wait gave up at site 0x%x", w[1]);
+        if (w[0] & kErrWaitTimeout)
+            snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "device wait gave up at site 0x%x", w[1]);
+        else
+            snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "a packed sequence is longer than max_seqlen");
         const unsigned int z[2] = {0, 0};
         e = cudaMemcpyToSymbol(g_error_word, z, sizeof(z));
         if (e != cudaSuccess) return cuda_fail(e);
-        return LA_ERR_TIMEOUT;
+        return (w[0] & kErrWaitTimeout) ? LA_ERR_TIMEOUT : LA_ERR_INVALID_ARG;
     }
     return LA_OK;
 }

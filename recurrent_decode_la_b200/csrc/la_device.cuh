@@ -16,7 +16,10 @@ namespace la {
 // ---------------------------------------------------------------------------
 extern __device__ unsigned int g_error_word[2];
 
-enum : unsigned int { kErrWaitTimeout = 1u };
+enum : unsigned int {
+    kErrWaitTimeout = 1u,  // a bounded wait gave up
+    kErrTooLong = 2u,      // a packed sequence longer than the max_seqlen promised
+};
 
 __device__ __forceinline__ void record_timeout(unsigned int where) {
     atomicOr(&g_error_word[0], kErrWaitTimeout);

@@ -76,6 +76,12 @@ cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap&
 // for s = 0 .. seg_count - 1 (one pass over the sub-segment sums).
 cudaError_t launch_segment_prefix(const PrefillProblem& p, float* seg_states, cudaStream_t s);
 
+// Prefill of at most kShortMaxTokens tokens per unit (dense T, or packed
+// max_seqlen) from a saved state: one pass over the state, CUDA cores, fp32.
+constexpr int kShortMaxTokens = 16;
+bool prefill_short_supported(int64_t max_tokens, int dk, int dv, const void* state);
+cudaError_t launch_prefill_short(const PrefillProblem& p, int64_t max_tokens, int num_sms, cudaStream_t s);
+
 // order[r] = the sequence of rank r when sequences are sorted by decreasing
 // length (ties: lower index first), for num_seqs <= kMaxOrderedSeqs.
 constexpr int kMaxOrderedSeqs = 4096;

@@ -1,0 +1,285 @@
+// la_prefill_short.cu -- prefill of a few tokens per unit (T <= 16) from a
+// saved state: the multi-token form of decode.
+//
+// With the whole input as one chunk of T tokens that starts from state S
+// (slides "Chunking, causality, and parallel prefill": "Causal triangle",
+// "Incoming and outgoing state"):
+//     o_t = q_t^T S + sum_{j <= t} (q_t . k_j) v_j,    S' = S + sum_t k_t v_t^T
+// Like a decode step, the cost is one read and one write of the fp32 state;
+// the T tokens only add T (d_k + d_v) inputs.  The d_v columns of a unit's
+// state may be split over CB CTAs when there are fewer units than SMs (o_t[j]
+// needs column j only, so there is no reduction across CTAs).  A CTA first
+// puts its whole state tile in flight with asynchronous copies into shared
+// memory (the bytes in flight are then not limited by registers), stages
+// q and k transposed (a row's tokens contiguous) and v, then each thread
+// takes four adjacent columns and a strided set of rows: it accumulates
+// q_t^T S of its columns for every token t in registers and writes the
+// updated rows straight back.  All arithmetic is fp32.
+#include <cuda_bf16.h>
+
+#include "la_device.cuh"
+#include "la_internal.h"
+
+namespace la {
+
+namespace {
+
+constexpr int kShortThreads = 256;
+constexpr int kShortWarps = kShortThreads / 32;
+
+template <typename E>
+__device__ __forceinline__ float elem_in(const E* p, int64_t i);
+template <>
+__device__ __forceinline__ float elem_in<float>(const float* p, int64_t i) {
+    return p[i];
+}
+template <>
+__device__ __forceinline__ float elem_in<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
+    return __bfloat162float(p[i]);
+}
+template <typename E>
+__device__ __forceinline__ void elem_out(E* p, int64_t i, float x);
+template <>
+__device__ __forceinline__ void elem_out<float>(float* p, int64_t i, float x) {
+    p[i] = x;
+}
+template <>
+__device__ __forceinline__ void elem_out<__nv_bfloat16>(__nv_bfloat16* p, int64_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ void fma4(float4& a, float s, const float4& b) {
+    a.x = fmaf(s, b.x, a.x);
+    a.y = fmaf(s, b.y, a.y);
+    a.z = fmaf(s, b.z, a.z);
+    a.w = fmaf(s, b.w, a.w);
+}
+
+// Shared memory (floats) of one CTA: the CTA's state tile [d_k][ncol], q
+// and k transposed [d_k][TM] (a row's tokens are contiguous), v [TM][ncol],
+// the causal scores [TM][TM], per-warp partial outputs [warps][TM][ncol].
+__host__ __device__ constexpr size_t short_smem_floats(int tm, int dk, int ncol) {
+    return static_cast<size_t>(dk) * ncol + 2 * static_cast<size_t>(dk) * tm +
+           static_cast<size_t>(tm) * ((1 + kShortWarps) * ncol + tm);
+}
+
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+
+template <typename E, int TM>
+__global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const PrefillProblem p, int cb_count) {
+    extern __shared__ float4 sm4[];
+    float* sm = reinterpret_cast<float*>(sm4);
+    const int dk = p.dk, dv = p.dv;
+    const int64_t u = blockIdx.x / cb_count;
+    const int ncol = dv / cb_count;
+    const int cbeg = static_cast<int>(blockIdx.x % cb_count) * ncol;
+    const int cols4 = ncol >> 2;
+    const int rpp = kShortThreads / cols4;  // rows per pass
+    const int tid = threadIdx.x;
+    const int c4 = tid % cols4;
+    const int r0 = tid / cols4;
+
+    // this unit's rows: dense unit u = group u, rows 0..T-1; packed unit
+    // n*H + h = head h, rows cu[n] .. cu[n+1]-1 (offsets out of range: empty)
+    int64_t group = u, row0 = 0;
+    int len;
+    if (p.cu == nullptr) {
+        len = static_cast<int>(p.rows_per_group);
+    } else {
+        const int n = static_cast<int>(u / p.H);
+        group = u % p.H;
+        const int a = p.cu[n], b = p.cu[n + 1];
+        const bool bad = a < 0 || b < a || static_cast<int64_t>(b) > p.rows_per_group;
+        row0 = bad ? 0 : a;
+        len = bad ? 0 : b - a;
+    }
+    if (len == 0) return;
+    if (len > TM) {
+        // longer than the max_seqlen the caller promised: leave the unit
+        // untouched and report it
+        if (tid == 0) atomicOr(&g_error_word[0], kErrTooLong);
+        return;
+    }
+    float* St = sm;                   // [dk][ncol]
+    float* qT = St + dk * ncol;       // [dk][TM]
+    float* kT = qT + dk * TM;         // [dk][TM]
+    float* vs = kT + dk * TM;         // [TM][ncol]
+    float* qk = vs + TM * ncol;       // [TM][TM]
+    float* red = qk + TM * TM;        // [warps][TM][ncol]
+    const int64_t rbase = group * p.rows_per_group + row0;
+    const E* Q = static_cast<const E*>(p.q) + rbase * dk;
+    const E* K = static_cast<const E*>(p.k) + rbase * dk;
+    const E* V = static_cast<const E*>(p.v) + rbase * dv;
+    E* O = static_cast<E*>(p.o) + rbase * dv;
+    float* Sg = p.state + u * static_cast<int64_t>(dk) * dv + cbeg;
+
+    // launched as a programmatic dependent of the previous kernel in the
+    // stream: nothing is read from global memory before it has finished
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the CTA's whole state tile goes in flight first (async copies into
+    // shared memory, no registers held)
+    for (int i = tid; i < dk * cols4; i += kShortThreads) {
+        const int r = i / cols4, c = i % cols4;
+        cp_async16(St + r * ncol + 4 * c, Sg + static_cast<int64_t>(r) * dv + 4 * c);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int i = tid; i < len * dk; i += kShortThreads) {
+        const int t = i / dk, r = i % dk;
+        qT[r * TM + t] = elem_in<E>(Q, i);
+        kT[r * TM + t] = elem_in<E>(K, i);
+    }
+    for (int i = tid; i < (TM - len) * dk; i += kShortThreads) {  // tokens past the end: zero
+        const int t = len + i / dk, r = i % dk;
+        qT[r * TM + t] = 0.f;
+        kT[r * TM + t] = 0.f;
+    }
+    for (int i = tid; i < TM * ncol; i += kShortThreads) {
+        const int t = i / ncol, c = i % ncol;
+        vs[i] = t < len ? elem_in<E>(V, static_cast<int64_t>(t) * dv + cbeg + c) : 0.f;
+    }
+    __syncthreads();
+    // causal scores q_t . k_j, j <= t (diagonal kept, the rest exactly 0)
+    for (int i = tid; i < TM * TM; i += kShortThreads) {
+        const int t = i / TM, j = i % TM;
+        float a = 0.f;
+        if (t < len && j <= t)
+            for (int r = 0; r < dk; ++r) a = fmaf(qT[r * TM + t], kT[r * TM + j], a);
+        qk[i] = a;
+    }
+    float4 vv[TM];
+#pragma unroll
+    for (int t = 0; t < TM; ++t) vv[t] = reinterpret_cast<const float4*>(vs + t * ncol)[c4];
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    // state pass: acc[t] += q_t[r] S[r][cols], then S[r] += sum_t k_t[r] v_t
+    // (tokens past the end have q = k = v = 0 and change nothing)
+    float4 acc[TM];
+#pragma unroll
+    for (int t = 0; t < TM; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int r = r0; r < dk; r += rpp) {
+        float4 s = reinterpret_cast<const float4*>(St + r * ncol)[c4];
+        const float4* q4 = reinterpret_cast<const float4*>(qT + r * TM);
+        const float4* k4 = reinterpret_cast<const float4*>(kT + r * TM);
+#pragma unroll
+        for (int t4 = 0; t4 < TM / 4; ++t4) {
+            const float4 qq = q4[t4];
+            fma4(acc[4 * t4 + 0], qq.x, s);
+            fma4(acc[4 * t4 + 1], qq.y, s);
+            fma4(acc[4 * t4 + 2], qq.z, s);
+            fma4(acc[4 * t4 + 3], qq.w, s);
+        }
+#pragma unroll
+        for (int t4 = 0; t4 < TM / 4; ++t4) {
+            const float4 kk = k4[t4];
+            fma4(s, kk.x, vv[4 * t4 + 0]);
+            fma4(s, kk.y, vv[4 * t4 + 1]);
+            fma4(s, kk.z, vv[4 * t4 + 2]);
+            fma4(s, kk.w, vv[4 * t4 + 3]);
+        }
+        reinterpret_cast<float4*>(Sg + static_cast<int64_t>(r) * dv)[c4] = s;
+    }
+    // sum the q_t^T S partials of the rows: lanes that own the same columns
+    // (shuffles), then the warps (shared memory)
+    const int lane = tid & 31, wid = tid >> 5;
+#pragma unroll
+    for (int t = 0; t < TM; ++t) {
+        for (int off = cols4; off < 32; off <<= 1) {
+            acc[t].x += __shfl_xor_sync(0xffffffffu, acc[t].x, off);
+            acc[t].y += __shfl_xor_sync(0xffffffffu, acc[t].y, off);
+            acc[t].z += __shfl_xor_sync(0xffffffffu, acc[t].z, off);
+            acc[t].w += __shfl_xor_sync(0xffffffffu, acc[t].w, off);
+        }
+        if (lane < cols4) reinterpret_cast<float4*>(red + (wid * TM + t) * ncol)[lane] = acc[t];
+    }
+    __syncthreads();
+    // o_t = q_t^T S + sum_{j <= t} (q_t . k_j) v_j
+    for (int i = tid; i < len * ncol; i += kShortThreads) {
+        const int t = i / ncol, c = i % ncol;
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kShortWarps; ++w) sum += red[(w * TM + t) * ncol + c];
+        for (int j = 0; j <= t; ++j) sum = fmaf(qk[t * TM + j], vs[j * ncol + c], sum);
+        elem_out<E>(O, static_cast<int64_t>(t) * dv + cbeg + c, sum);
+    }
+}
+
+// Column blocks per unit: the fewest (so that each CTA stages a large state
+// tile) that still give every SM a CTA, each block a whole number of float4
+// columns whose count divides the block's threads.  0 when d_v does not
+// allow it.
+int short_col_blocks(int64_t n_units, int num_sms, int dv) {
+    auto ok = [&](int cb) {
+        if (dv % (4 * cb) != 0) return false;
+        const int cols4 = dv / (4 * cb);
+        return cols4 <= 32 && kShortThreads % cols4 == 0;
+    };
+    if (!ok(1)) return 0;
+    int cb = 1;
+    while (cb < 8 && n_units * cb < num_sms && ok(cb * 2)) cb *= 2;
+    return cb;
+}
+
+template <typename E, int TM>
+cudaError_t launch_short_tm(const PrefillProblem& p, int cb, cudaStream_t s) {
+    auto kern = prefill_short_kernel<E, TM>;
+    const size_t smem = short_smem_floats(TM, p.dk, p.dv / cb) * sizeof(float);
+    // raise the limit to the largest this instantiation can ask for, once
+    // per device (not inside a stream capture: the first launch sets it)
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(short_smem_floats(TM, 128, 128) * sizeof(float)));
+        if (e != cudaSuccess) return e;
+        // all of the SM's unified L1/shared storage as shared memory, so that
+        // two CTAs with large state tiles can be resident together
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.n_units * cb), 1, 1);
+    cfg.blockDim = dim3(kShortThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, p, cb);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <typename E>
+cudaError_t launch_short_t(const PrefillProblem& p, int64_t max_tokens, int cb, cudaStream_t s) {
+    if (max_tokens <= 4) return launch_short_tm<E, 4>(p, cb, s);
+    if (max_tokens <= 8) return launch_short_tm<E, 8>(p, cb, s);
+    return launch_short_tm<E, 16>(p, cb, s);
+}
+
+}  // namespace
+
+bool prefill_short_supported(int64_t max_tokens, int dk, int dv, const void* state) {
+    return max_tokens >= 1 && max_tokens <= kShortMaxTokens && dk >= 1 && dk <= 128 && dv >= 4 && dv <= 128 &&
+           (reinterpret_cast<uintptr_t>(state) & 15) == 0 && short_col_blocks(1, 1, dv) > 0;
+}
+
+cudaError_t launch_prefill_short(const PrefillProblem& p, int64_t max_tokens, int num_sms, cudaStream_t s) {
+    if (p.n_units <= 0) return cudaSuccess;
+    const int cb = short_col_blocks(p.n_units, num_sms, p.dv);
+    if (cb == 0 || p.n_units * cb > 2147483647LL) return cudaErrorInvalidValue;
+    return p.dtype == 1 ? launch_short_t<__nv_bfloat16>(p, max_tokens, cb, s)
+                        : launch_short_t<float>(p, max_tokens, cb, s);
+}
+
+}  // namespace la

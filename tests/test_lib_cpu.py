@@ -47,6 +47,14 @@ def test_kernel_choice():
     assert la.la_prefill_path(torch.bfloat16, 64, 64, 16) == "tc"
     assert la.la_prefill_path(torch.bfloat16, 128, 128, 48) == "simt"
     assert la.la_prefill_path(torch.bfloat16, 96, 96, 64) == "simt"
+    # with the token count: at most 16 tokens per unit run the few-token kernel
+    assert la.la_prefill_kernel(torch.bfloat16, 16, 128, 128) == "short"
+    assert la.la_prefill_kernel(torch.float32, 1, 5, 8) == "short"
+    assert la.la_prefill_kernel(torch.bfloat16, 17, 128, 128) == "tc"
+    assert la.la_prefill_kernel(torch.float32, 17, 128, 128) == "simt"
+    assert la.la_prefill_kernel(torch.bfloat16, 8, 128, 6) == "simt"     # d_v not a multiple of 4
+    assert la.la_prefill_kernel(torch.bfloat16, 8, 128, 80) == "simt"    # 20 float4 columns do not split 256 threads
+    assert la.la_prefill_kernel(torch.bfloat16, 0, 128, 128) == "tc"     # packed, max_seqlen unknown
     assert la.la_prefill_path(torch.float32, 128, 128, 64) == "simt"
     assert la.la_prefill_path(torch.float32, 2, 2, 4) == "simt"
     assert la.la_prefill_path(torch.bfloat16, 256, 256, 64) == "unsupported"
