@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-short", action="store_true", help="skip the few-token prefill measurement")
+    ap.add_argument("--short-only", type=int, default=0, metavar="UNITS",
+                    help="only the few-token prefill measurement, on UNITS units (multiple of 32) of the workload's d")
     ap.add_argument("--no-cold-decode", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the oracle sample")
@@ -797,6 +799,24 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
             "h2d_gbs": h2d / (ms / n_steps * 1e-3) / 1e9}
 
 
+def run_short_only(args, wl):
+    """Only the few-token prefill measurement (8 tokens per unit, cold
+    state) on args.short_only units of 32 heads; prints one JSON line."""
+    import torch
+
+    import recurrent_decode_la_b200 as la
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    la.load_library()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    H = 32
+    B = max(1, args.short_only // H)
+    res = short_prefill(la, torch, dev, stream, wl, B, H, 8, peaks, peak_src)
+    print(json.dumps({"short_prefill": res, "device_status": la.la_status_string(la.la_device_status(stream))}))
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     from recurrent_decode_la_b200 import inputs
@@ -807,6 +827,8 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, wl, world, rank)
+    if args.short_only:
+        return run_short_only(args, wl)
     if wl.varlen:
         return run_varlen(args, wl, world, rank, local)
     return run_ours(args, wl, world, rank, local)
