@@ -1,5 +1,5 @@
 // la_device.cuh -- sm_100a device helpers: mbarriers with bounded waits,
-// TMA tile copies (no multicast), tcgen05 MMA / TMEM access, shared-memory
+// TMA tile copies (each CTA loads its own tiles), tcgen05 MMA / TMEM access, shared-memory
 // matrix descriptors.  Inline PTX only; no library kernels.
 #pragma once
 
@@ -125,7 +125,7 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 }
 
 // ---------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), tile mode, never multicast.
+// TMA (cp.async.bulk.tensor), tile mode; every copy targets this CTA's shared memory only.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
