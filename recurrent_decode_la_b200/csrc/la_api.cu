@@ -310,7 +310,8 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
         // Packed sequences, more units than SMs: the persistent CTAs claim
         // units from a counter (so lengths that differ, and SMs that run at
         // different speeds, even out), longest sequences first.
-        if (cu_seqlens && n_units > sms && workspace && workspace_bytes >= 256 && aligned16(workspace)) {
+        if (cu_seqlens && n_units > sms && n_units < 0x7fffffffLL && workspace && workspace_bytes >= 256 &&
+            aligned16(workspace)) {
             unsigned int* counter = static_cast<unsigned int*>(workspace);
             e = cudaMemsetAsync(counter, 0, sizeof(unsigned int), s);
             if (e != cudaSuccess) return cuda_fail(e);
