@@ -6,7 +6,31 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace la {
+
+// Per-device one-time set-up of a kernel's attributes (a raised shared-memory
+// limit and the like).  cudaFuncSetAttribute may not run inside a stream
+// capture, so the first launch on each device (made outside any capture)
+// runs it; later launches skip it.  Safe to call from several host threads:
+// the attribute calls are idempotent, the flags atomic.  Devices beyond the
+// first 64 run the set-up on every launch.
+struct PerDeviceOnce {
+    std::atomic<bool> done[64];  // static storage: zero-initialised
+    template <typename F>
+    cudaError_t run(F&& setup) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        const bool cached = dev >= 0 && dev < 64;
+        if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        e = setup();
+        if (e != cudaSuccess) return e;
+        if (cached) done[dev].store(true, std::memory_order_release);
+        return cudaSuccess;
+    }
+};
 
 // Everything a prefill kernel needs to locate its units.  Dense input:
 // groups = B*H, rows_per_group = T, unit u = group u.  Packed input:

@@ -231,20 +231,16 @@ cudaError_t launch_short_tm(const PrefillProblem& p, int cb, cudaStream_t s) {
     const size_t smem = short_smem_floats(TM, p.dk, p.dv / cb) * sizeof(float);
     // raise the limit to the largest this instantiation can ask for, once
     // per device (not inside a stream capture: the first launch sets it)
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(short_smem_floats(TM, 128, 128) * sizeof(float)));
-        if (e != cudaSuccess) return e;
+    static PerDeviceOnce attrs;
+    cudaError_t e = attrs.run([&] {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(short_smem_floats(TM, 128, 128) * sizeof(float)));
+        if (r != cudaSuccess) return r;
         // all of the SM's unified L1/shared storage as shared memory, so that
         // two CTAs with large state tiles can be resident together
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
+        return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(p.n_units * cb), 1, 1);
     cfg.blockDim = dim3(kShortThreads, 1, 1);

@@ -1104,15 +1104,10 @@ static cudaError_t launch_sub_impl(const PrefillProblem& p, const CUtensorMap& t
                                    float* sub_states, int num_sms, cudaStream_t s) {
     using Cfg = KvCfg<C, D>;
     auto kern = subsegment_states_kernel<C, D>;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static PerDeviceOnce attrs;
+    cudaError_t e = attrs.run(
+        [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM); });
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
     const int64_t items = p.n_units * p.subs_per_unit;
     const int64_t grid = items < num_sms ? items : num_sms;
     if (grid < 1) return cudaSuccess;
@@ -1208,15 +1203,10 @@ static cudaError_t launch_tc_impl(const PrefillProblem& p, const CUtensorMap& tq
     auto kern = prefill_tc_kernel<C, D>;
     // Raise the dynamic shared-memory limit once per device (not inside a
     // stream capture: the first launch on a device sets it).
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static PerDeviceOnce attrs;
+    cudaError_t e = attrs.run(
+        [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM); });
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
     const int64_t items = p.n_units * p.seg_count;
     int64_t grid = items < num_sms ? items : num_sms;
     if (grid < 1) return cudaSuccess;
