@@ -99,3 +99,24 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 4, 8)
     with pytest.raises(ValueError):
         la.la_prefill(x, x, x, x.clone(), torch.zeros(1, 8, 8))
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No CPU fallback: with the shared library absent, the first call raises."""
+    code = (
+        "import os, sys\n"
+        f"os.environ['LINATTN_LIB'] = {str(tmp_path / 'absent.so')!r}\n"
+        "import recurrent_decode_la_b200 as la\n"
+        "try:\n"
+        "    la.la_status_string(0)\n"
+        "except OSError as e:\n"
+        "    print('raised', e)\n"
+        "    sys.exit(0)\n"
+        "sys.exit(1)\n"
+    )
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "absent.so" in r.stdout
