@@ -306,7 +306,8 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     if (path == kTc) {
         CUtensorMap tq, tk, tv, to;
         if (!encode_bf16_map(&tq, q, d_k, T, groups, c) || !encode_bf16_map(&tk, k, d_k, T, groups, c) ||
-            !encode_bf16_map(&tv, v, d_v, T, groups, c) || !encode_bf16_map(&to, o, d_v, T, groups, c)) {
+            !encode_bf16_map(&tv, v, d_v, T, groups, c) ||
+            !encode_bf16_map(&to, o, d_v, T, groups, prefill_tc_o_box_rows(c))) {
             snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed");
             return LA_ERR_CUDA;
         }

@@ -86,6 +86,9 @@ size_t prefill_simt_smem_bytes(int dk, int dv, int chunk);
 
 // Tensor-core prefill (bf16, d_k == d_v == D in {64,128}, chunk in {16,32,64,128}).
 bool prefill_tc_supported(int D, int chunk);
+// Rows of the O tensor map's box for this chunk size (C = 128: each output
+// warp stores its own 32 rows).
+int prefill_tc_o_box_rows(int chunk);
 cudaError_t launch_prefill_tc(const PrefillProblem& p, const CUtensorMap& tq,
                               const CUtensorMap& tk, const CUtensorMap& tv,
                               const CUtensorMap& to, int num_sms, cudaStream_t s);

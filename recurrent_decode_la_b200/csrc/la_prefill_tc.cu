@@ -185,8 +185,9 @@ __global__ void __launch_bounds__(512, 1)
         for (int s = 0; s < Cfg::NS; ++s) {
             mbar_init(&bar[Cfg::B_FULL + s], 1);
             // released by the state stream's K^T V and by the chunk's last
-            // other reader (the P V MMA, or the O store that reuses Q's tile)
-            mbar_init(&bar[Cfg::B_EMPTY + s], 2);
+            // other reader: the P V MMA, or (C = 128) the O stores that reuse
+            // the Q tile, one per output warp
+            mbar_init(&bar[Cfg::B_EMPTY + s], Cfg::PT ? 5 : 2);
             mbar_init(&bar[Cfg::B_ZERO + s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -861,24 +862,32 @@ __global__ void __launch_bounds__(512, 1)
                     __syncwarp();
                     if (lane == 0) {
                         mbar_arrive(&bar[Cfg::B_OEMPTY + ob]);
-                        mbar_arrive(&bar[Cfg::B_OSTFULL + osb]);
+                        if (!Cfg::PT) mbar_arrive(&bar[Cfg::B_OSTFULL + osb]);
                         if (warp == 12) LA_TRACE(31, g);
                     }
-                    if (elected) {
+                    if constexpr (Cfg::PT) {
+                        // each warp stores its own 32 rows as soon as they are
+                        // staged (the O tensor map's box is 32 rows high here)
+                        // and hands its share of the stage back once the
+                        // store has read them
+                        if (lane == 0) {
+#pragma unroll
+                            for (int pn = 0; pn < Cfg::NPAN; ++pn)
+                                tma_store_3d(&tmO, smem + (stg - sbase) + pn * Cfg::PANEL + sub * 32 * 128, pn * 64,
+                                             un.row0 + c * C + sub * 32, un.group);
+                            bulk_commit_group();
+                            bulk_wait_group_read<0>();
+                            mbar_arrive(&bar[Cfg::B_EMPTY + st_s]);
+                        }
+                    } else if (elected) {
                         if (mbar_wait(&bar[Cfg::B_OSTFULL + osb], (f / 2) & 1, abort_flag, tmo, 0x420 + osb)) {
 #pragma unroll
                             for (int pn = 0; pn < Cfg::NPAN; ++pn)
                                 tma_store_3d(&tmO, smem + (stg - sbase) + pn * Cfg::PANEL, pn * 64,
                                              un.row0 + c * C, un.group);
                             bulk_commit_group();
-                            if constexpr (Cfg::PT) {
-                                // the stage returns to the producer once the store has read it
-                                bulk_wait_group_read<0>();
-                                mbar_arrive(&bar[Cfg::B_EMPTY + st_s]);
-                            } else {
-                                bulk_wait_group_read<1>();
-                                if (f >= 1) mbar_arrive(&bar[Cfg::B_OSTFREE + ((f - 1) & 1)]);
-                            }
+                            bulk_wait_group_read<1>();
+                            if (f >= 1) mbar_arrive(&bar[Cfg::B_OSTFREE + ((f - 1) & 1)]);
                         }
                     }
                     ++f;
@@ -905,11 +914,11 @@ __global__ void __launch_bounds__(512, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bar[Cfg::B_OEMPTY + ob]);
-                    if (Cfg::PT && elected) mbar_arrive(&bar[Cfg::B_EMPTY + st_s]);
+                    if (Cfg::PT && lane == 0) mbar_arrive(&bar[Cfg::B_EMPTY + st_s]);
                 }
             }
         }
-        if (elected) bulk_wait_group<0>();
+        if (lane == 0) bulk_wait_group<0>();  // every output warp's stores have landed
     }
 
     tc_fence_before();
@@ -1190,6 +1199,8 @@ cudaError_t launch_length_order(const int32_t* cu, int num_seqs, int64_t total_r
     length_order_kernel<<<(num_seqs + threads - 1) / threads, threads, 0, s>>>(cu, num_seqs, total_rows, order);
     return cudaGetLastError();
 }
+
+int prefill_tc_o_box_rows(int chunk) { return chunk == 128 ? 32 : chunk; }
 
 bool prefill_tc_supported(int D, int chunk) {
     return (D == 64 || D == 128) && (chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128);
