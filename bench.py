@@ -234,6 +234,18 @@ def _oracle_units_for(wl, seconds, dsteps):
     return min(n_units, rounds * len(probe)), cores
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or "" if unknown."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
 def run_reference(args, wl, world, rank):
     """The reference arm: the float64 CPU oracle (C recurrence over OpenMP
     threads) timed on a bounded sample of the same workload."""
@@ -263,7 +275,7 @@ def run_reference(args, wl, world, rank):
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "T": wl.T, "d_k": wl.d, "d_v": wl.d,
                    "decode_steps": dsteps, "sample_units": units, "of_units": n_units},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -276,7 +288,7 @@ def cpu_baseline_sample(wl, seconds, dsteps):
     units, cores = _oracle_units_for(wl, seconds, dsteps)
     t = _oracle_pass(wl, list(range(units)), dsteps)
     tokens = units * (wl.T + dsteps) / wl.H
-    return {"value": tokens / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    return {"value": tokens / t, "unit": "tokens/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{units} of {inputs.n_units(wl)} (sequence, head) units: full T={wl.T} prefill + "
                       f"{dsteps} decode tokens each, float64 recurrence, {t:.1f} s; tokens = unit rows / H"}
 
