@@ -11,7 +11,8 @@ import torch
 import recurrent_decode_la_b200 as la
 from oracle import la_oracle as ora
 from recurrent_decode_la_b200 import inputs
-from gpu_util import BF16_TOL, F32_TOL, gpu_prefill, nerr, oracle_units
+from gpu_util import (BF16_TOL, F32_TOL, decode_tokens, decode_vs_oracle, gpu_decode_run, gpu_prefill, nerr,
+                      prefill_vs_oracle)
 
 pytestmark = pytest.mark.gpu
 
@@ -238,77 +239,86 @@ def test_prefill_then_decode_equals_longer_prefill():
 
 
 # ------------------------------------------- the five workloads ----
+#
+# Every unit of every workload is compared with the oracle (streamed over
+# batches of units), and decode runs every step on every unit, starting from
+# the oracle's own prefill states: the errors below cover the whole path,
+# prefill then decode.  Outputs start as NaN, so a unit or step the kernels
+# skipped fails.
 
-def _decode_run(wl, S_dev, units, steps, sample):
-    """Run `steps` decode steps on all `units` states; oracle on `sample` units."""
-    Sd = S_dev.reshape(units, wl.d, wl.d)
-    Sr = {u: Sd[u].double().cpu().numpy() for u in sample}
-    worst = 0.0
-    for step in range(steps):
-        q, k, v = inputs.decode_token(wl, step, units=units)
-        od = torch.empty(units, 1, wl.d, dtype=wl.torch_dtype, device="cuda")
-        la.la_decode_step(q.cuda()[:, None], k.cuda()[:, None], v.cuda()[:, None], od, Sd)
-        oc = od.float().cpu()
-        for u in sample:
-            o_ref, Sr[u] = ora.decode_step(q[u], k[u], v[u], Sr[u])
-            worst = max(worst, nerr(oc[u, 0], o_ref))
-    Sc = Sd.cpu()
-    worst_s = max(nerr(Sc[u], Sr[u]) for u in sample)
-    return worst, worst_s
+def _report(name, **errs):
+    print(f"{name}: " + ", ".join(f"{k}={v:.3e}" if isinstance(v, float) else f"{k}={v}" for k, v in errs.items()))
+
+
+def _assert_ok(errs, tol):
+    for e in errs if isinstance(errs, list) else [errs]:
+        assert e["nonfinite"] == 0, e
+        for key, val in e.items():
+            if key != "nonfinite":
+                assert val <= tol, e
 
 
 def test_workload_b4h8_t2048_d64_full():
     wl = WL["b4h8_t2048_d64"]
     q, k, v, _ = inputs.prefill_inputs(wl)
     assert la.la_prefill_path(wl.torch_dtype, wl.d, wl.d, wl.chunk) == "tc"
-    O_ref, S_ref = ora.recurrent(q, k, v)
     o, S = gpu_prefill(q, k, v, chunk=wl.chunk)
-    assert nerr(o, O_ref) <= BF16_TOL
-    assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
-    e_o, e_s = _decode_run(wl, S, inputs.decode_units(wl), wl.decode_steps, sample=[0, 13, 31])
-    assert e_o <= BF16_TOL and e_s <= BF16_TOL
+    (e,), S_ref = prefill_vs_oracle(q, k, v, [(o, S)])
+    units = inputs.decode_units(wl)
+    dq, dk_, dv = decode_tokens(wl, wl.decode_steps, units)
+    od = gpu_decode_run(S.reshape(units, wl.d, wl.d), dq, dk_, dv)
+    ed = decode_vs_oracle(dq, dk_, dv, od, S, S_ref)
+    _report(wl.name, prefill_O=e["O"], prefill_S=e["S"], decode_o=ed["o"], decode_S=ed["S"])
+    _assert_ok([e, ed], BF16_TOL)
 
 
-@pytest.mark.parametrize("chunk", [32, 64, 128])
-def test_workload_b8h16_t8192_d128_sampled(chunk):
+def test_workload_b8h16_t8192_d128_all_units():
+    """All 128 units at C = 32, 64 and 128 (one oracle pass for the three),
+    then the full 256 decode steps on all 128 states from C = 128 (the bench's
+    default) and from C = 64 (the workload's listed chunk)."""
     wl = WL["b8h16_t8192_d128_knorm"]
     q, k, v, _ = inputs.prefill_inputs(wl)
-    o, S = gpu_prefill(q, k, v, chunk=chunk)
-    assert torch.isfinite(o).all() and torch.isfinite(S).all()
-    sample = [0, 37, 64, 127]
-    for u, (O_ref, S_ref) in zip(sample, oracle_units(wl, sample)):
-        b, h = divmod(u, wl.H)
-        assert nerr(o[b, h], O_ref) <= BF16_TOL, u
-        assert nerr(S[u], S_ref) <= BF16_TOL, u
-    if chunk == 64:
-        e_o, e_s = _decode_run(wl, S, inputs.decode_units(wl), 32, sample=[0, 77])
-        assert e_o <= BF16_TOL and e_s <= BF16_TOL
+    runs = {c: gpu_prefill(q, k, v, chunk=c) for c in (32, 64, 128)}
+    errs, S_ref = prefill_vs_oracle(q, k, v, list(runs.values()))
+    for c, e in zip(runs, errs):
+        _report(f"{wl.name} C={c}", prefill_O=e["O"], prefill_S=e["S"])
+    units = inputs.decode_units(wl)
+    dq, dk_, dv = decode_tokens(wl, wl.decode_steps, units)
+    dec = {}
+    for c in (128, 64):
+        S = runs[c][1].reshape(units, wl.d, wl.d)
+        od = gpu_decode_run(S, dq, dk_, dv)
+        dec[c] = decode_vs_oracle(dq, dk_, dv, od, S, S_ref)
+        _report(f"{wl.name} decode after C={c}", decode_o=dec[c]["o"], decode_S=dec[c]["S"])
+    _assert_ok(errs + list(dec.values()), BF16_TOL)
 
 
-def test_workload_b1h32_t131072_d128_sampled():
+def test_workload_b1h32_t131072_d128_all_units():
+    """All 32 units of the long sequences (the split into segments is taken:
+    32 units on a GPU of more than 64 SMs)."""
     wl = WL["b1h32_t131072_d128"]
     q, k, v, _ = inputs.prefill_inputs(wl)
     o, S = gpu_prefill(q, k, v, chunk=wl.chunk)
-    assert torch.isfinite(S).all()
-    sample = [0, 31]
-    for u, (O_ref, S_ref) in zip(sample, oracle_units(wl, sample)):
-        assert nerr(o[0, u], O_ref) <= BF16_TOL, u
-        assert nerr(S[u], S_ref) <= BF16_TOL, u
+    (e,), _ = prefill_vs_oracle(q, k, v, [(o, S)])
+    _report(wl.name, prefill_O=e["O"], prefill_S=e["S"])
+    _assert_ok(e, BF16_TOL)
 
 
-def test_workload_varlen64_h32_d128_sampled():
+def test_workload_varlen64_h32_d128_all_units():
+    """All 2048 packed (sequence, head) units, then the 64 x 32 final states
+    repeated 4 times -> 256 x 32 decode units, all 512 steps on all of them."""
     wl = WL["varlen64_h32_d128"]
     q, k, v, cu = inputs.prefill_inputs(wl)
     lens = (cu[1:] - cu[:-1]).numpy()
     o, S = gpu_prefill(q, k, v, cu=cu, chunk=wl.chunk, max_seqlen=int(lens.max()))
-    assert torch.isfinite(S).all()
-    sample = [0, 5 * wl.H + 7, int(np.argmax(lens)) * wl.H + 31, int(np.argmin(lens)) * wl.H + 2]
-    for u, (O_ref, S_ref) in zip(sample, oracle_units(wl, sample)):
-        h, r0, L = inputs.unit_rows(wl, u)
-        assert nerr(o[0, h, r0:r0 + L], O_ref) <= BF16_TOL, u
-        assert nerr(S.reshape(-1, wl.d, wl.d)[u], S_ref) <= BF16_TOL, u
-    # decode: the 64 x 32 prefilled states, repeated 4 times -> 256 x 32 units
+    (e,), S_ref = prefill_vs_oracle(q, k, v, [(o, S)], cu=cu.numpy())
+    _report(wl.name, prefill_O=e["O"], prefill_S=e["S"])
+    del o, q, k, v
     units = inputs.decode_units(wl)
     Sdec = S.reshape(-1, wl.d, wl.d).repeat(wl.decode_repeat, 1, 1).contiguous()
-    e_o, e_s = _decode_run(wl, Sdec, units, 16, sample=[0, units - 1])
-    assert e_o <= BF16_TOL and e_s <= BF16_TOL
+    S_ref_dec = np.tile(S_ref, (wl.decode_repeat, 1, 1))
+    dq, dk_, dv = decode_tokens(wl, wl.decode_steps, units)
+    od = gpu_decode_run(Sdec, dq, dk_, dv)
+    ed = decode_vs_oracle(dq, dk_, dv, od, Sdec, S_ref_dec)
+    _report(f"{wl.name} decode", decode_o=ed["o"], decode_S=ed["S"])
+    _assert_ok([e, ed], BF16_TOL)

@@ -8,7 +8,8 @@ no workspace and draws the scratch of the intra-sequence split from a static
 buffer inside the library.  This test calls it through the C ABI twice in a
 row -- the second call reuses a buffer still holding the first call's data --
 and checks each result against la_prefill given a caller-allocated workspace,
-within the bf16 tolerance the other parity tests use.
+and every unit of it against the float64 oracle, within the bf16 tolerance
+the other parity tests use.
 
 Kept in a file of its own, collected last, so that a run stopping at the
 first failure has already run every other test.
@@ -20,7 +21,7 @@ import pytest
 import torch
 
 import recurrent_decode_la_b200 as la
-from gpu_util import BF16_TOL, nerr
+from gpu_util import BF16_TOL, nerr, prefill_vs_oracle
 from recurrent_decode_la_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -50,7 +51,8 @@ def test_noalloc_prefill_matches_prefill_twice(lib):
     for seed, (B, H, T, d, chunk) in enumerate([(1, 4, 8192, 128, 128), (1, 8, 3000, 128, 64)]):
         need = la.la_prefill_workspace_size(torch.bfloat16, B, H, T, d, d, 0, chunk)
         assert 0 < need <= 64 * 1024 * 1024
-        q, k, v = (x.to(dev) for x in inputs.random_qkv(100 + seed, B, H, T, d, d, dtype=torch.bfloat16))
+        q_h, k_h, v_h = inputs.random_qkv(100 + seed, B, H, T, d, d, dtype=torch.bfloat16)
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
         S0 = torch.from_numpy(
             np.random.default_rng(seed).standard_normal((B * H, d, d)).astype(np.float32) * 0.05).to(dev)
 
@@ -60,8 +62,8 @@ def test_noalloc_prefill_matches_prefill_twice(lib):
         ws = torch.empty(need, dtype=torch.uint8, device=dev)
         la.la_prefill(q, k, v, o_ref, st_ref, chunk=chunk, workspace=ws)
 
-        # the entry point that allocates nothing
-        o = torch.empty_like(v)
+        # the entry point that allocates nothing (output NaN until written)
+        o = torch.full_like(v, float("nan"))
         st = S0.clone()
         status = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), st.data_ptr(), la.LA_BF16,
                     B, H, T, d, d, None, 0, 0, chunk, stream)
@@ -70,3 +72,5 @@ def test_noalloc_prefill_matches_prefill_twice(lib):
 
         assert nerr(o, o_ref.float().cpu().numpy()) <= BF16_TOL
         assert nerr(st, st_ref.cpu().numpy()) <= BF16_TOL
+        (e,), _ = prefill_vs_oracle(q_h, k_h, v_h, [(o, st)], S0=S0.cpu().numpy())
+        assert e["nonfinite"] == 0 and e["O"] <= BF16_TOL and e["S"] <= BF16_TOL, e
