@@ -111,6 +111,8 @@ def _check(status: int, where: str) -> None:
 def la_state_init(state: torch.Tensor, src: Optional[torch.Tensor] = None,
                   stream=None) -> None:
     """state [..., d_k, d_v] float32 <- src (or zero)."""
+    if state.dim() < 2:
+        raise ValueError("state must be [..., d_k, d_v]")
     dk, dv = state.shape[-2], state.shape[-1]
     n = state.numel() // max(1, dk * dv)
     if src is not None and src.shape != state.shape:
@@ -134,15 +136,27 @@ def la_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tenso
     [B,H,d_k,d_v] (or [N,H,d_k,d_v] with cu_seqlens, B == 1)."""
     if q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {q.dtype}")
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, T, d_k]")
     B, H, T, dk = q.shape
     dv = v.shape[-1]
-    if k.shape != q.shape or v.shape[:3] != q.shape[:3] or o.shape != v.shape:
+    if k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3] or o.shape != v.shape:
         raise ValueError("q/k/v/o shapes disagree")
     num_seqs = 0
     if cu_seqlens is not None:
         if cu_seqlens.dtype != torch.int32:
             raise ValueError("cu_seqlens must be int32")
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must hold num_seqs + 1 >= 2 offsets")
+        if B != 1:
+            raise ValueError("packed input (cu_seqlens) needs B == 1")
         num_seqs = cu_seqlens.numel() - 1
+    # the kernels read and write n_units * d_k * d_v floats of state: a smaller
+    # buffer would be overrun, so its size is checked here, before any launch
+    n_units = (num_seqs if cu_seqlens is not None else B) * H
+    if state.numel() != n_units * dk * dv:
+        raise ValueError(f"state must hold {n_units} x {dk} x {dv} floats "
+                         f"({'num_seqs' if cu_seqlens is not None else 'B'} * H units), got {state.numel()}")
     ws_ptr, ws_bytes = None, 0
     if workspace is not None:
         ws_ptr, ws_bytes = _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size()
@@ -159,10 +173,14 @@ def la_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.T
     [B,H,d_k,d_v] updated in place."""
     if q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {q.dtype}")
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H, d_k]")
     B, H, dk = q.shape
     dv = v.shape[-1]
-    if k.shape != q.shape or v.shape[:2] != q.shape[:2] or o.shape != v.shape:
+    if k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2] or o.shape != v.shape:
         raise ValueError("q/k/v/o shapes disagree")
+    if state.numel() != B * H * dk * dv:
+        raise ValueError(f"state must hold {B * H} x {dk} x {dv} floats, got {state.numel()}")
     _check(load_library().la_decode_step(
         _ptr(q, "q", q.dtype), _ptr(k, "k", q.dtype), _ptr(v, "v", q.dtype),
         _ptr(o, "o", q.dtype), _ptr(state, "state", torch.float32), _DTYPES[q.dtype],

@@ -120,3 +120,28 @@ def test_missing_library_fails_loudly(tmp_path):
                        cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     assert r.returncode == 0, r.stdout + r.stderr
     assert "absent.so" in r.stdout
+
+
+@pytest.mark.parametrize("case", ["small_state", "dense_state_for_packed", "short_cu", "packed_b2", "decode_state"])
+def test_binding_checks_state_size_before_any_launch(case):
+    """The kernels read and write units * d_k * d_v floats of state; the
+    binding refuses a state of another size (and malformed packed offsets)
+    with ValueError, before it touches the library or the device."""
+    d = 8
+    x = torch.zeros(2, 3, 5, d)
+    with pytest.raises(ValueError):
+        if case == "small_state":
+            la.la_prefill(x, x, x, x.clone(), torch.zeros(2 * 3 - 1, d, d))
+        elif case == "dense_state_for_packed":
+            xp = torch.zeros(1, 3, 10, d)
+            cu = torch.tensor([0, 4, 7, 10], dtype=torch.int32)           # 3 sequences x 3 heads
+            la.la_prefill(xp, xp, xp, xp.clone(), torch.zeros(1 * 3, d, d), cu_seqlens=cu)
+        elif case == "short_cu":
+            xp = torch.zeros(1, 3, 10, d)
+            la.la_prefill(xp, xp, xp, xp.clone(), torch.zeros(3, d, d), cu_seqlens=torch.tensor([0], dtype=torch.int32))
+        elif case == "packed_b2":
+            cu = torch.tensor([0, 5], dtype=torch.int32)
+            la.la_prefill(x, x, x, x.clone(), torch.zeros(1 * 3, d, d), cu_seqlens=cu)
+        else:
+            t = torch.zeros(2, 3, d)
+            la.la_decode_step(t, t, t, t.clone(), torch.zeros(2 * 3, d, d - 1))
