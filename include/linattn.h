@@ -79,7 +79,8 @@ la_status la_state_init(float* state, const float* src, int64_t n_units,
  *     most 16 the few-token kernel runs, and a sequence too long for it is
  *     left untouched and reported by la_device_status (LA_ERR_INVALID_ARG).
  *   chunk: C, the number of tokens per chunk; 0 picks the default for the
- *     shape (LINATTN_CHUNK in the environment overrides the default).
+ *     shape (LINATTN_CHUNK in the environment overrides the default; like
+ *     every LINATTN_* switch it is read once per process, on first use).
  *   workspace / workspace_bytes: device scratch of la_prefill_workspace_size()
  *     bytes, 16-byte aligned, owned by the caller and free for the library
  *     until the call's work on `stream` has finished.  It buys speed only:
@@ -124,7 +125,9 @@ size_t la_prefill_workspace_size(la_dtype dtype, int B, int H, int64_t T,
  * the library.  Nothing is allocated or freed, by this call or any library it
  * calls.
  *   - The first call on a device looks up that device's address of the
- *     buffer; make that first call before any stream capture.
+ *     buffer (again when the device's current context has changed, e.g.
+ *     after cudaDeviceReset); make that first call before any stream
+ *     capture.
  *   - Every call on a device shares the one buffer, and calls that overlap
  *     on the GPU (different streams, no ordering between them) race on it.
  *     Every byte a call reads from the buffer was written earlier in the same

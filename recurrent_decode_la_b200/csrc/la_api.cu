@@ -21,6 +21,36 @@ namespace la {
 
 __device__ unsigned int g_error_word[2];
 
+const Tuning& tuning() {
+    // C++ guarantees this initialiser runs once, even with concurrent callers.
+    static const Tuning t = [] {
+        auto get = [](const char* name) -> const char* {
+            const char* e = getenv(name);
+            return e && *e ? e : nullptr;
+        };
+        Tuning v;
+        const char* e = get("LINATTN_CHUNK");
+        v.chunk = e ? atoi(e) : 0;
+        e = get("LINATTN_SHORT");
+        v.short_kernel = !(e && e[0] == '0');
+        e = get("LINATTN_SPLIT");
+        v.split = !(e && e[0] == '0');
+        e = get("LINATTN_PREFETCH");
+        v.prefetch = e ? atoi(e) : 1;  // one chunk ahead: measured best on B200 (deeper thrashes L2)
+        if (v.prefetch < 0) v.prefetch = 0;
+        e = get("LINATTN_DECODE_COLBLOCKS");
+        v.decode_col_blocks = e ? atoi(e) : -1;
+        e = get("LINATTN_DECODE_PDL");
+        v.decode_pdl = !(e && e[0] == '0');
+        e = get("LINATTN_WAIT_TIMEOUT_MS");
+        double ms = e ? atof(e) : 4000.0;
+        if (!(ms > 0)) ms = 4000.0;
+        v.wait_timeout_ns = static_cast<uint64_t>(ms * 1e6);
+        return v;
+    }();
+    return t;
+}
+
 namespace {
 
 thread_local char g_last_cuda_error[256] = "";
@@ -45,16 +75,6 @@ int current_sm_count() {
     return n;
 }
 
-uint64_t wait_timeout_ns() {
-    static uint64_t v = [] {
-        const char* e = getenv("LINATTN_WAIT_TIMEOUT_MS");
-        double ms = e ? atof(e) : 4000.0;
-        if (!(ms > 0)) ms = 4000.0;
-        return static_cast<uint64_t>(ms * 1e6);
-    }();
-    return v;
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -66,6 +86,23 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     });
     return fn;
+}
+
+// The calling thread's current CUDA context (nullptr if the driver entry
+// point cannot be found or no context is current).
+CUcontext current_context() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    });
+    CUcontext c = nullptr;
+    if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
 }
 
 // 3-D bf16 view (d, rows, groups) of a [groups][rows][d] tensor, box
@@ -85,11 +122,7 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, int d, int64_t rows, in
 }
 
 int default_chunk(la_dtype dtype, int dk, int dv) {
-    const char* e = getenv("LINATTN_CHUNK");
-    if (e) {
-        const int c = atoi(e);
-        if (c > 0) return c;
-    }
+    if (tuning().chunk > 0) return tuning().chunk;
     // bf16 tensor-core path: 128-token chunks run full-rate M = 128 MMAs with
     // P kept in tensor memory (the measured fastest chunk on B200).
     if (dtype == LA_BF16 && dk == dv && (dk == 64 || dk == 128)) return 128;
@@ -122,8 +155,7 @@ struct SplitPlan {
 SplitPlan plan_split(int64_t n_units, int64_t T, int dk, int dv, int chunk, int sms) {
     SplitPlan sp;
     sp.seg_len = T;
-    const char* e = getenv("LINATTN_SPLIT");
-    if (e && e[0] == '0') return sp;
+    if (!tuning().split) return sp;
     if (n_units <= 0 || T <= 0) return sp;
     const int64_t nch = (T + chunk - 1) / chunk;
     int64_t P = sms / n_units;
@@ -175,8 +207,7 @@ Path choose_path(la_dtype dtype, int dk, int dv, int chunk, const void* q, const
 Path choose_kernel(la_dtype dtype, int64_t max_tokens, int dk, int dv, int chunk, const void* q, const void* k,
                    const void* v, const void* o, const void* state) {
     if (dk < 1 || dv < 1 || dk > 128 || dv > 128 || chunk < 1) return kUnsupported;
-    const char* e = getenv("LINATTN_SHORT");
-    if (!(e && e[0] == '0') && prefill_short_supported(max_tokens, dk, dv, state)) return kShort;
+    if (tuning().short_kernel && prefill_short_supported(max_tokens, dk, dv, state)) return kShort;
     Path path = choose_path(dtype, dk, dv, chunk, q, k, v, o);
     // The tensor-core kernel moves state rows with 16-byte accesses.
     if (path == kTc && !aligned16(state)) path = kSimt;
@@ -279,7 +310,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     p.dk = d_k; p.dv = d_v;
     p.cu = cu_seqlens;
     p.chunk = c;
-    p.timeout_ns = wait_timeout_ns();
+    p.timeout_ns = tuning().wait_timeout_ns;
     p.seg_count = 1;
     p.seg_len = T;
     p.sub_len = 0;
@@ -289,10 +320,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, float
     p.seg_states = nullptr;
     p.work_counter = nullptr;
     p.order = nullptr;
-    {
-        const char* pf = getenv("LINATTN_PREFETCH");
-        p.prefetch = pf ? atoi(pf) : 1;  // measured best on B200 (deeper prefetch thrashes)
-    }
+    p.prefetch = tuning().prefetch;
     p.trace = g_trace.buf;
     p.trace_count = g_trace.count;
     p.trace_cap = g_trace.cap;
@@ -397,19 +425,24 @@ la_status la_prefill_noalloc(const void* q, const void* k, const void* v, void* 
     void* scratch = nullptr;
     if (need > 0) {
         // Device address of the static buffer, looked up once per device
-        // with that device current.
+        // with that device current, and again whenever the device's current
+        // context is no longer the one it was looked up in (after a
+        // cudaDeviceReset, say, the old address is stale).
         static void* addr[64] = {nullptr};
+        static CUcontext ctx_of[64] = {nullptr};
         static std::mutex mu;
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return cuda_fail(e);
         if (dev < 0 || dev >= 64) return LA_ERR_UNSUPPORTED;
+        const CUcontext ctx = current_context();  // nullptr before the runtime has made one current
         std::lock_guard<std::mutex> lock(mu);
-        if (!addr[dev]) {
+        if (!addr[dev] || ctx == nullptr || ctx != ctx_of[dev]) {
             void* ptr = nullptr;
-            e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+            e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);  // makes the primary context current
             if (e != cudaSuccess) return cuda_fail(e);
             addr[dev] = ptr;
+            ctx_of[dev] = current_context();
         }
         scratch = addr[dev];
     }

@@ -5,14 +5,14 @@
 // is 1x1 and only the state read plus the local term remain):
 //     S' = S + k v^T,        o = q^T S'   ( = q^T S + (q . k) v )
 // The step reads the fp32 state once and writes it once, so it is bound by
-// memory bandwidth.  A block owns one unit: each thread owns four adjacent
-// columns of the state and a strided set of its rows, issues all of its
-// 128-bit state loads before any arithmetic (so they are in flight
-// together), updates the rows, stores them back, and keeps a partial
-// q^T S' for its columns; the partials of the rows are summed in shared
+// memory bandwidth.  The main kernel splits a unit's d_v columns over a few
+// CTAs (o[j] only needs column j of S', so no reduction crosses CTAs); each
+// thread owns four adjacent columns and a strided set of rows, has all of
+// its 128-bit state loads in flight before any arithmetic, updates the rows,
+// stores them back, and keeps a partial q^T S' for its columns; the partials
+// of the rows are summed by warp shuffles, then across warps in shared
 // memory.
 #include <cuda_bf16.h>
-#include <stdlib.h>
 
 #include "la_internal.h"
 
@@ -37,6 +37,11 @@ __device__ __forceinline__ void dec_out<float>(float* p, int64_t i, float x) {
 template <>
 __device__ __forceinline__ void dec_out<__nv_bfloat16>(__nv_bfloat16* p, int64_t i, float x) {
     p[i] = __float2bfloat16_rn(x);
+}
+
+// Bring the 128-byte line holding p into L2 (a hint: no data is returned).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
 }
 
 constexpr int kDecThreads = 256;
@@ -104,40 +109,63 @@ __global__ void __launch_bounds__(kDecThreads) decode_vec_kernel(const T* __rest
 
 // Column-split form: the d_v columns of a unit's state are split over CB
 // CTAs, each of which owns all d_k rows of its columns, so o[j] (a sum over
-// rows of column j) needs no reduction across CTAs.  With a few hundred units
-// this still fills every SM and keeps more loads in flight per SM.  Launched
-// as a programmatic dependent of the previous kernel in the stream: a CTA may
-// start while that kernel drains, but reads nothing from global memory before
-// griddepcontrol.wait returns.
-template <typename T, int NR>
-__global__ void __launch_bounds__(kDecThreads, 4) decode_cols_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                                     const T* __restrict__ v, T* __restrict__ o,
-                                                                     float* __restrict__ state, int64_t n_units,
-                                                                     int dk, int dv, int cb_count) {
+// rows of column j) needs no reduction across CTAs.
+//
+// Launched as a programmatic dependent of the previous kernel in the stream.
+// A CTA may start while that kernel still runs: before griddepcontrol.wait it
+// only prefetches its state rows and its q, k, v into L2, and it reads
+// nothing before the wait returns.  A prefetch is a hint that moves no data
+// into registers or shared memory, and L2 is the device's point of coherence
+// for global memory, so a line the previous kernel writes after the prefetch
+// is still read correctly after the wait.  The prefetch takes the HBM
+// latency of the state off the critical path of a chain of decode launches
+// (one per layer, say).  At most 32 registers per thread (eight 256-thread
+// CTAs per SM) leave room for the next launch's CTAs to become resident, and
+// prefetch, while this launch runs.
+//
+// FDK / FNC fix d_k = d_v and the columns per CTA at compile time (0: taken
+// from the arguments).  The fixed forms (d 64 or 128, 16 or 32 columns) fit
+// in 32 registers; the general form runs four CTAs per SM.
+template <typename T, int NR, int FDK, int FNC>
+__global__ void __launch_bounds__(kDecThreads, (FDK > 0 ? 8 : 4))
+    decode_cols_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
+                       float* __restrict__ state, int64_t n_units, int dk_arg, int dv_arg, int cb_count) {
     extern __shared__ float sm[];
     float* qs = sm;
     float* ks = qs + 128;
     float* vs = ks + 128;
-    float* red = vs + 128;  // [rows per pass][cols of this CTA]
+    float* red = vs + 128;  // [warps][cols of this CTA]
+    const int dk = FDK > 0 ? FDK : dk_arg;
+    const int dv = FDK > 0 ? FDK : dv_arg;
     const int64_t u = blockIdx.x / cb_count;
     const int cb = static_cast<int>(blockIdx.x % cb_count);
-    const int ncol = dv / cb_count;        // columns of this CTA
+    const int ncol = FNC > 0 ? FNC : dv / cb_count;  // columns of this CTA
     const int cbeg = cb * ncol;
     const int cols4 = ncol >> 2;
     const int rpp = kDecThreads / cols4;   // rows per pass
     const int tid = threadIdx.x;
     const int c4 = tid % cols4;
     const int r0 = tid / cols4;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     float4* S = reinterpret_cast<float4*>(state + u * static_cast<int64_t>(dk) * dv + cbeg) + c4;
     const int row4 = dv >> 2;  // float4 per state row
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int r = r0; r < dk; r += rpp) prefetch_l2(S + r * row4);
+    {
+        constexpr int kPer = 128 / static_cast<int>(sizeof(T));  // elements per 128-byte line
+        const int i = tid * kPer;
+        if (i < dk) {
+            prefetch_l2(q + u * dk + i);
+            prefetch_l2(k + u * dk + i);
+        }
+        if (i < ncol) prefetch_l2(v + u * dv + cbeg + i);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // first batch of this thread's rows: loads in flight before anything else
     float4 sv[NR];
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
         const int r = r0 + i * rpp;
-        if (r < dk) sv[i] = S[r * row4];
+        if (FDK > 0 || r < dk) sv[i] = S[r * row4];
     }
     for (int i = tid; i < dk; i += kDecThreads) {
         qs[i] = dec_in<T>(q, u * dk + i);
@@ -147,6 +175,25 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_cols_kernel(const T* __
     __syncthreads();
     const float4 vv = make_float4(vs[4 * c4], vs[4 * c4 + 1], vs[4 * c4 + 2], vs[4 * c4 + 3]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (FDK > 0) {
+        // fixed form: NR rows per thread cover d_k exactly, one batch
+        static_assert(NR * (kDecThreads / (FNC / 4)) == FDK, "rows per thread");
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const int r = r0 + i * rpp;
+            const float kr = ks[r], qr = qs[r];
+            float4 s4 = sv[i];
+            s4.x = fmaf(kr, vv.x, s4.x);
+            s4.y = fmaf(kr, vv.y, s4.y);
+            s4.z = fmaf(kr, vv.z, s4.z);
+            s4.w = fmaf(kr, vv.w, s4.w);
+            S[r * row4] = s4;
+            acc.x = fmaf(qr, s4.x, acc.x);
+            acc.y = fmaf(qr, s4.y, acc.y);
+            acc.z = fmaf(qr, s4.z, acc.z);
+            acc.w = fmaf(qr, s4.w, acc.w);
+        }
+    } else
 #pragma unroll 1
     for (int rb = 0; r0 + rb * rpp < dk; rb += NR) {
         if (rb > 0) {
@@ -235,11 +282,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_scalar_kernel(const T* __r
     }
 }
 
-static int env_int(const char* name, int dflt) {
-    const char* e = getenv(name);
-    return e && *e ? atoi(e) : dflt;
-}
-
 template <typename T>
 static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* state, int64_t n_units, int dk,
                                int dv, int cb, cudaStream_t s) {
@@ -252,25 +294,38 @@ static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* 
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = env_int("LINATTN_DECODE_PDL", 1) ? 1 : 0;
-    // rows per thread held in registers at once (batches of up to 4): few
-    // registers, so four 256-thread CTAs stay resident per SM
-    const int rpp = kDecThreads / (dv / (4 * cb));
+    cfg.numAttrs = tuning().decode_pdl ? 1 : 0;
+    const int ncol = dv / cb;
+    const bool sq = (dk == dv);
+    if (sq && dk == 128 && ncol == 32)
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 4, 128, 32>, q, k, v, o, state, n_units, dk, dv, cb);
+    if (sq && dk == 128 && ncol == 16)
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 2, 128, 16>, q, k, v, o, state, n_units, dk, dv, cb);
+    if (sq && dk == 64 && ncol == 32)
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 2, 64, 32>, q, k, v, o, state, n_units, dk, dv, cb);
+    if (sq && dk == 64 && ncol == 16)
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 1, 64, 16>, q, k, v, o, state, n_units, dk, dv, cb);
+    // other shapes: rows per thread held in registers at once, batches of up to 4
+    const int rpp = kDecThreads / (ncol / 4);
     const int need = (dk + rpp - 1) / rpp;
-    if (need <= 1) return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 1>, q, k, v, o, state, n_units, dk, dv, cb);
-    if (need <= 2) return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 2>, q, k, v, o, state, n_units, dk, dv, cb);
-    return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 4>, q, k, v, o, state, n_units, dk, dv, cb);
+    if (need <= 1)
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 1, 0, 0>, q, k, v, o, state, n_units, dk, dv, cb);
+    if (need <= 2)
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 2, 0, 0>, q, k, v, o, state, n_units, dk, dv, cb);
+    return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 4, 0, 0>, q, k, v, o, state, n_units, dk, dv, cb);
 }
 
-// Column blocks per unit: enough CTAs to cover the SMs about three times,
-// each block a whole number of float4 columns, at most 16 rows per thread.
+// Column blocks per unit: 32 columns per CTA where d_v allows it (each row
+// piece one 128-byte line; measured best on B200 from 128 to 8192 units),
+// more blocks while the grid covers the SMs less than about three times.
+// Every block is a whole number of float4 columns.
 static int decode_col_blocks(int64_t n_units, int num_sms, int dk, int dv) {
     auto ok = [&](int cb) {
-        if (dv % (4 * cb) != 0) return false;
+        if (cb < 1 || dv % (4 * cb) != 0) return false;
         const int cols4 = dv / (4 * cb);
         return kDecThreads % cols4 == 0;
     };
-    int cb = 1;
+    int cb = (dv % 32 == 0 && ok(dv / 32)) ? dv / 32 : 1;
     while (cb < 8 && n_units * cb < 3LL * num_sms && ok(cb * 2)) cb *= 2;
     return ok(cb) ? cb : 0;
 }
@@ -284,12 +339,11 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     const bool vec = (dv % 4 == 0) && cols4 > 0 && (kDecThreads % cols4 == 0) &&
                      (reinterpret_cast<uintptr_t>(state) % 16 == 0) &&
                      ((dk + (kDecThreads / cols4) - 1) / (kDecThreads / cols4) <= kDecMaxRowsPerThread);
-    // 2^31 CTAs at most; the cluster form needs n_units * CL of them.
-    // LINATTN_DECODE_COLBLOCKS overrides the column split (0 = one CTA per unit
+    // The column split launches n_units * cb CTAs (2^31 at most).
+    // LINATTN_DECODE_COLBLOCKS overrides the split (0 = one CTA per unit,
     // without a programmatic launch).
     int cb = (vec && n_units <= (1LL << 27)) ? decode_col_blocks(n_units, num_sms, dk, dv) : 0;
-    const int force = env_int("LINATTN_DECODE_COLBLOCKS", -1);
-    if (vec && force >= 0) cb = force;
+    if (vec && tuning().decode_col_blocks >= 0) cb = tuning().decode_col_blocks;
     if (cb > 0 && (dv % (4 * cb) != 0 || kDecThreads % (dv / (4 * cb)) != 0)) cb = 0;
     if (cb > 0) {
         cudaError_t e;

@@ -10,6 +10,29 @@
 
 namespace la {
 
+// Tuning switches taken from the environment once per process, on the first
+// call into the library that needs one; later changes to the environment
+// have no effect.  None of them changes a result, only which kernel runs or
+// how it is scheduled.
+//   LINATTN_CHUNK             default chunk size (0 / unset: per shape)
+//   LINATTN_SHORT=0           never take the few-token prefill kernel
+//   LINATTN_SPLIT=0           never split a sequence into segments
+//   LINATTN_PREFETCH          chunks the prefill producer prefetches into L2
+//   LINATTN_DECODE_COLBLOCKS  decode column blocks per unit (unset: per
+//                             shape; 0: one CTA per unit)
+//   LINATTN_DECODE_PDL=0      launch decode without programmatic dependency
+//   LINATTN_WAIT_TIMEOUT_MS   bound of every device-side wait (default 4000)
+struct Tuning {
+    int chunk;
+    bool short_kernel;
+    bool split;
+    int prefetch;
+    int decode_col_blocks;  // -1: per shape
+    bool decode_pdl;
+    uint64_t wait_timeout_ns;
+};
+const Tuning& tuning();
+
 // Per-device one-time set-up of a kernel's attributes (a raised shared-memory
 // limit and the like).  cudaFuncSetAttribute may not run inside a stream
 // capture, so the first launch on each device (made outside any capture)

@@ -2,50 +2,16 @@
 one CTA per unit, scalar), decode at thousands of units, and the fp32
 CUDA-core prefill with d_k != d_v and odd sizes.  Each compares the CUDA path
 with the float64 oracle on the same seeded inputs."""
-import os
-
 import numpy as np
 import pytest
 import torch
 
 import recurrent_decode_la_b200 as la
-from gpu_util import BF16_TOL, F32_TOL, gpu_prefill, nerr, tol_for
+from gpu_util import BF16_TOL, F32_TOL, decode_steps_vs_oracle, gpu_prefill, nerr, run_in_child, tol_for
 from oracle import la_oracle as ora
 from recurrent_decode_la_b200 import inputs
 
 pytestmark = pytest.mark.gpu
-
-
-def _decode_steps(dtype, B, H, dk, dv, steps, seed, env=None):
-    """Run `steps` decode tokens from a random state through la_decode_step;
-    return (gpu outputs, gpu final state, oracle outputs, oracle final state)."""
-    rng = np.random.default_rng(seed)
-    S0 = (rng.standard_normal((B, H, dk, dv)) * 0.05).astype(np.float32)
-    toks = [inputs.random_qkv(seed * 100 + i, B, H, 1, dk, dv, dtype=dtype) for i in range(steps)]
-    st = torch.from_numpy(S0).cuda()
-    outs = []
-    old = {kk: os.environ.get(kk) for kk in (env or {})}
-    try:
-        os.environ.update(env or {})
-        for q, k, v in toks:
-            o = torch.empty(B, H, dv, dtype=dtype, device="cuda")
-            la.la_decode_step(q[:, :, 0].contiguous().cuda(), k[:, :, 0].contiguous().cuda(),
-                              v[:, :, 0].contiguous().cuda(), o, st)
-            outs.append(o)
-        assert la.la_device_status() == la.LA_OK
-    finally:
-        for kk, vv in old.items():
-            if vv is None:
-                os.environ.pop(kk, None)
-            else:
-                os.environ[kk] = vv
-    S = S0.astype(np.float64)
-    refs = []
-    for q, k, v in toks:
-        o_ref, S = ora.decode_step(q[:, :, 0].float().numpy(), k[:, :, 0].float().numpy(),
-                                   v[:, :, 0].float().numpy(), S)
-        refs.append(o_ref)
-    return torch.stack(outs), st, np.stack(refs), S
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -59,10 +25,16 @@ def _decode_steps(dtype, B, H, dk, dv, steps, seed, env=None):
     (128, 6, None),
 ])
 def test_decode_kernels(dtype, dk, dv, env):
-    outs, st, refs, S = _decode_steps(dtype, 2, 3, dk, dv, 4, seed=dk * 7 + dv, env=env)
+    """Each decode kernel against the oracle; a kernel chosen through an
+    environment switch runs in a child process (switches are read once per
+    process)."""
+    if env:
+        errs = run_in_child("decode", env, dtype="bf16" if dtype == torch.bfloat16 else "f32",
+                            dk=dk, dv=dv, steps=4, seed=dk * 7 + dv)
+    else:
+        errs = decode_steps_vs_oracle(dtype, 2, 3, dk, dv, 4, seed=dk * 7 + dv)
     tol = tol_for(dtype)
-    assert nerr(outs, refs) <= tol
-    assert nerr(st.reshape(S.shape), S) <= tol
+    assert errs["o"] <= tol and errs["S"] <= tol, errs
 
 
 def test_decode_8192_units_sampled():

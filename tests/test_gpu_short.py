@@ -3,14 +3,12 @@ multi-token form of decode) against the float64 oracle: dense and packed
 layouts, both dtypes, d_k != d_v, empty sequences, a sequence longer than the
 promised max_seqlen (reported, its unit left untouched), agreement with the
 chunked kernels, and prefill + short continuation == one longer prefill."""
-import os
-
 import numpy as np
 import pytest
 import torch
 
 import recurrent_decode_la_b200 as la
-from gpu_util import BF16_TOL, F32_TOL, gpu_prefill, nerr, tol_for
+from gpu_util import BF16_TOL, F32_TOL, gpu_prefill, nerr, run_in_child, tol_for
 from oracle import la_oracle as ora
 from recurrent_decode_la_b200 import inputs
 
@@ -82,20 +80,21 @@ def test_short_sequence_longer_than_promised_is_reported():
 
 
 def test_short_matches_chunked_kernels():
-    B, H, T, d = 2, 8, 16, 128
-    q, k, v = inputs.random_qkv(21, B, H, T, d, d, dtype=torch.bfloat16)
-    S0 = _state(4, B, H, d, d)
+    """The same 16-token prefill through the few-token kernel and, in a child
+    process started with LINATTN_SHORT=0, through the chunked tensor-core
+    kernel: both match the oracle."""
+    B, H, T, d, seed = 2, 8, 16, 128, 21
+    assert la.la_prefill_kernel(torch.bfloat16, T, d, d) == "short"
+    res = {"short": None, "tc": run_in_child("prefill", {"LINATTN_SHORT": "0"}, dtype="bf16", B=B, H=H, T=T, d=d,
+                                             seed=seed)}
+    assert res["tc"]["kernel"] == "tc"
+    q, k, v = inputs.random_qkv(seed, B, H, T, d, d, dtype=torch.bfloat16)
+    S0 = torch.from_numpy((np.random.default_rng(seed).standard_normal((B, H, d, d)) * 0.05).astype(np.float32))
     O_ref, S_ref = ora.recurrent(q, k, v, S0)
-    o1, S1 = gpu_prefill(q, k, v, S0=S0)
-    os.environ["LINATTN_SHORT"] = "0"
-    try:
-        assert la.la_prefill_kernel(torch.bfloat16, T, d, d) == "tc"
-        o2, S2 = gpu_prefill(q, k, v, S0=S0)
-    finally:
-        os.environ.pop("LINATTN_SHORT", None)
-    for o, S in ((o1, S1), (o2, S2)):
-        assert nerr(o, O_ref) <= BF16_TOL
-        assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
+    o, S = gpu_prefill(q, k, v, S0=S0)
+    res["short"] = {"o": nerr(o, O_ref), "S": nerr(S.reshape(S_ref.shape), S_ref)}
+    for name, e in res.items():
+        assert e["o"] <= BF16_TOL and e["S"] <= BF16_TOL, (name, e)
 
 
 def test_prefill_then_short_continuation_equals_longer_prefill():
