@@ -63,6 +63,11 @@ __host__ __device__ constexpr size_t short_smem_floats(int tm, int dk, int ncol)
            static_cast<size_t>(tm) * ((1 + kShortWarps) * ncol + tm);
 }
 
+// Bring the 128-byte line holding p into L2 (a hint: no data is returned).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                  "l"(src)
@@ -117,9 +122,26 @@ __global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const P
     E* O = static_cast<E*>(p.o) + rbase * dv;
     float* Sg = p.state + u * static_cast<int64_t>(dk) * dv + cbeg;
 
-    // launched as a programmatic dependent of the previous kernel in the
-    // stream: nothing is read from global memory before it has finished
+    // Launched as a programmatic dependent of the previous kernel in the
+    // stream: nothing is read from global memory before griddepcontrol.wait
+    // returns.  Before it, the CTA only prefetches its state tile and its
+    // tokens into L2 (a hint; L2 is the point of coherence, so a line the
+    // previous kernel writes afterwards is still read correctly), which takes
+    // the HBM latency off the chain of a sequence of such calls.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int i = tid; i < dk * ((ncol + 31) / 32); i += kShortThreads) {
+        const int r = i / ((ncol + 31) / 32), c = (i % ((ncol + 31) / 32)) * 32;
+        prefetch_l2(Sg + static_cast<int64_t>(r) * dv + c);
+    }
+    {
+        constexpr int kPer = 128 / static_cast<int>(sizeof(E));  // elements per 128-byte line
+        const int nq = len * dk, nv = len * dv;
+        for (int i = tid * kPer; i < nq; i += kShortThreads * kPer) {
+            prefetch_l2(Q + i);
+            prefetch_l2(K + i);
+        }
+        for (int i = tid * kPer; i < nv; i += kShortThreads * kPer) prefetch_l2(V + i);
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the CTA's whole state tile goes in flight first (async copies into
     // shared memory, no registers held)
@@ -128,19 +150,29 @@ __global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const P
         cp_async16(St + r * ncol + 4 * c, Sg + static_cast<int64_t>(r) * dv + 4 * c);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    for (int i = tid; i < len * dk; i += kShortThreads) {
-        const int t = i / dk, r = i % dk;
-        qT[r * TM + t] = elem_in<E>(Q, i);
-        kT[r * TM + t] = elem_in<E>(K, i);
-    }
-    for (int i = tid; i < (TM - len) * dk; i += kShortThreads) {  // tokens past the end: zero
-        const int t = len + i / dk, r = i % dk;
-        qT[r * TM + t] = 0.f;
-        kT[r * TM + t] = 0.f;
-    }
-    for (int i = tid; i < TM * ncol; i += kShortThreads) {
-        const int t = i / ncol, c = i % ncol;
-        vs[i] = t < len ? elem_in<E>(V, static_cast<int64_t>(t) * dv + cbeg + c) : 0.f;
+    {
+        // every token load in flight before the first shared-memory store
+        // (d_k, d_v <= 128: at most TM / 2 elements of each per thread)
+        constexpr int kPer = (TM * 128 + kShortThreads - 1) / kShortThreads;
+        float qv[kPer], kv[kPer], vv[kPer];
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int i = tid + j * kShortThreads;
+            qv[j] = i < len * dk ? elem_in<E>(Q, i) : 0.f;
+            kv[j] = i < len * dk ? elem_in<E>(K, i) : 0.f;
+            const int t = i / ncol, c = i % ncol;
+            vv[j] = (i < TM * ncol && t < len) ? elem_in<E>(V, static_cast<int64_t>(t) * dv + cbeg + c) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int i = tid + j * kShortThreads;
+            if (i < TM * dk) {  // tokens past the end are zero
+                const int t = i / dk, r = i % dk;
+                qT[r * TM + t] = qv[j];
+                kT[r * TM + t] = kv[j];
+            }
+            if (i < TM * ncol) vs[i] = vv[j];
+        }
     }
     __syncthreads();
     // causal scores q_t . k_j, j <= t (diagonal kept, the rest exactly 0)
