@@ -145,3 +145,28 @@ def test_binding_checks_state_size_before_any_launch(case):
         else:
             t = torch.zeros(2, 3, d)
             la.la_decode_step(t, t, t, t.clone(), torch.zeros(2 * 3, d, d - 1))
+
+
+def test_tuning_switches_are_read_once():
+    """LINATTN_* switches are read on first use and never again: changing the
+    environment later in the process changes nothing (a captured graph and a
+    later direct call always agree)."""
+    code = (
+        "import os, sys\n"
+        "os.environ['LINATTN_CHUNK'] = '64'\n"
+        "import torch\n"
+        "import recurrent_decode_la_b200 as la\n"
+        "a = la.la_resolve_chunk(torch.bfloat16, 128, 128, 0)\n"
+        "os.environ['LINATTN_CHUNK'] = '32'\n"
+        "b = la.la_resolve_chunk(torch.bfloat16, 128, 128, 0)\n"
+        "del os.environ['LINATTN_CHUNK']\n"
+        "c = la.la_resolve_chunk(torch.bfloat16, 128, 128, 0)\n"
+        "print(a, b, c)\n"
+        "sys.exit(0 if (a, b, c) == (64, 64, 64) else 1)\n"
+    )
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if not k.startswith("LINATTN_")}
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, env=env,
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    assert r.returncode == 0, r.stdout + r.stderr
