@@ -127,10 +127,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_vec_kernel(const T* __rest
 // L2-resident step slower than four CTAs per SM.
 //
 // FDK / FNC fix d_k = d_v and the columns per CTA at compile time (0: taken
-// from the arguments): d 64 or 128 with 16 or 32 columns run one batch of
-// rows per thread with every index known to the compiler.
-template <typename T, int NR, int FDK, int FNC>
-__global__ void __launch_bounds__(kDecThreads, 4)
+// from the arguments): d 64 or 128 with 16, 32 or 64 columns run one batch of
+// rows per thread with every index known to the compiler.  NT threads per
+// CTA: 256 (four CTAs per SM), or 1024 for few units (fewer, larger CTAs
+// launch faster; each thread then holds two rows).
+template <typename T, int NR, int FDK, int FNC, int NT = kDecThreads>
+__global__ void __launch_bounds__(NT, (NT >= 1024 ? 1 : 4))
     decode_cols_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
                        float* __restrict__ state, int64_t n_units, int dk_arg, int dv_arg, int cb_count) {
     extern __shared__ float sm[];
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kDecThreads, 4)
     const int ncol = FNC > 0 ? FNC : dv / cb_count;  // columns of this CTA
     const int cbeg = cb * ncol;
     const int cols4 = ncol >> 2;
-    const int rpp = kDecThreads / cols4;   // rows per pass
+    const int rpp = NT / cols4;   // rows per pass
     const int tid = threadIdx.x;
     const int c4 = tid % cols4;
     const int r0 = tid / cols4;
@@ -170,17 +172,17 @@ __global__ void __launch_bounds__(kDecThreads, 4)
         const int r = r0 + i * rpp;
         if (FDK > 0 || r < dk) sv[i] = S[r * row4];
     }
-    for (int i = tid; i < dk; i += kDecThreads) {
+    for (int i = tid; i < dk; i += NT) {
         qs[i] = dec_in<T>(q, u * dk + i);
         ks[i] = dec_in<T>(k, u * dk + i);
     }
-    for (int i = tid; i < ncol; i += kDecThreads) vs[i] = dec_in<T>(v, u * dv + cbeg + i);
+    for (int i = tid; i < ncol; i += NT) vs[i] = dec_in<T>(v, u * dv + cbeg + i);
     __syncthreads();
     const float4 vv = make_float4(vs[4 * c4], vs[4 * c4 + 1], vs[4 * c4 + 2], vs[4 * c4 + 3]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (FDK > 0) {
         // fixed form: NR rows per thread cover d_k exactly, one batch
-        static_assert(NR * (kDecThreads / (FNC / 4)) == FDK, "rows per thread");
+        static_assert(NR * (NT / (FNC / 4)) == FDK, "rows per thread");
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
             const int r = r0 + i * rpp;
@@ -235,10 +237,10 @@ __global__ void __launch_bounds__(kDecThreads, 4)
     const int lane = tid & 31, wid = tid >> 5;
     if (lane < cols4) reinterpret_cast<float4*>(red + wid * ncol)[lane] = acc;
     __syncthreads();
-    for (int n = tid; n < ncol; n += kDecThreads) {
+    for (int n = tid; n < ncol; n += NT) {
         float sum = 0.f;
 #pragma unroll
-        for (int w = 0; w < kDecThreads / 32; ++w) sum += red[w * ncol + n];
+        for (int w = 0; w < NT / 32; ++w) sum += red[w * ncol + n];
         dec_out<T>(o, u * dv + cbeg + n, sum);
     }
 }
@@ -287,11 +289,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_scalar_kernel(const T* __r
 
 template <typename T>
 static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* state, int64_t n_units, int dk,
-                               int dv, int cb, cudaStream_t s) {
+                               int dv, int cb, bool big, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_units * cb), 1, 1);
-    cfg.blockDim = dim3(kDecThreads, 1, 1);
-    cfg.dynamicSmemBytes = sizeof(float) * (3 * 128 + 1024);
+    cfg.blockDim = dim3(big ? 1024 : kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = sizeof(float) * (3 * 128 + (big ? 32 * 64 : 1024));
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -300,6 +302,9 @@ static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* 
     cfg.numAttrs = tuning().decode_pdl ? 1 : 0;
     const int ncol = dv / cb;
     const bool sq = (dk == dv);
+    if (big)  // d = 128, two 1024-thread CTAs per unit, 64 columns each
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 2, 128, 64, 1024>, q, k, v, o, state, n_units, dk, dv,
+                                  cb);
     if (sq && dk == 128 && ncol == 32)
         return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 4, 128, 32>, q, k, v, o, state, n_units, dk, dv, cb);
     if (sq && dk == 128 && ncol == 16)
@@ -346,17 +351,27 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     // LINATTN_DECODE_COLBLOCKS overrides the split (0 = one CTA per unit,
     // without a programmatic launch).
     int cb = (vec && n_units <= (1LL << 27)) ? decode_col_blocks(n_units, num_sms, dk, dv) : 0;
-    if (vec && tuning().decode_col_blocks >= 0) cb = tuning().decode_col_blocks;
+    // Few units at d = 128: two 1024-thread CTAs per unit, when they fit in
+    // one wave of two CTAs per SM (measured on B200 at 128 units: 3.24 against
+    // 3.83 us per step with a cold state; at 1024 units and more the
+    // 256-thread form is faster).
+    bool big = vec && dk == 128 && dv == 128 && n_units * 2 <= 2LL * num_sms;
+    if (big) cb = 2;
+    if (vec && tuning().decode_col_blocks >= 0) {
+        cb = tuning().decode_col_blocks;
+        big = false;
+    }
     if (cb > 0 && (dv % (4 * cb) != 0 || kDecThreads % (dv / (4 * cb)) != 0)) cb = 0;
     if (cb > 0) {
         cudaError_t e;
         if (dtype == 0)
             e = launch_cols<float>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                   static_cast<const float*>(v), static_cast<float*>(o), state, n_units, dk, dv, cb, s);
+                                   static_cast<const float*>(v), static_cast<float*>(o), state, n_units, dk, dv, cb,
+                                   big, s);
         else
             e = launch_cols<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                            static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), state,
-                                           n_units, dk, dv, cb, s);
+                                           n_units, dk, dv, cb, big, s);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
