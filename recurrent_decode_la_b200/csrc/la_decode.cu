@@ -302,8 +302,11 @@ static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* 
     cfg.numAttrs = tuning().decode_pdl ? 1 : 0;
     const int ncol = dv / cb;
     const bool sq = (dk == dv);
-    if (big)  // d = 128, two 1024-thread CTAs per unit, 64 columns each
+    if (big && dk == 128)  // two 1024-thread CTAs per unit, 64 columns each
         return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 2, 128, 64, 1024>, q, k, v, o, state, n_units, dk, dv,
+                                  cb);
+    if (big)  // d = 64: one 1024-thread CTA per unit
+        return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 1, 64, 64, 1024>, q, k, v, o, state, n_units, dk, dv,
                                   cb);
     if (sq && dk == 128 && ncol == 32)
         return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 4, 128, 32>, q, k, v, o, state, n_units, dk, dv, cb);
@@ -351,12 +354,13 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     // LINATTN_DECODE_COLBLOCKS overrides the split (0 = one CTA per unit,
     // without a programmatic launch).
     int cb = (vec && n_units <= (1LL << 27)) ? decode_col_blocks(n_units, num_sms, dk, dv) : 0;
-    // Few units at d = 128: two 1024-thread CTAs per unit, when they fit in
-    // one wave of two CTAs per SM (measured on B200 at 128 units: 3.24 against
-    // 3.83 us per step with a cold state; at 1024 units and more the
-    // 256-thread form is faster).
-    bool big = vec && dk == 128 && dv == 128 && n_units * 2 <= 2LL * num_sms;
-    if (big) cb = 2;
+    // Few units: 1024-thread CTAs, two per unit at d = 128 and one at d = 64,
+    // when they fit in one wave of two CTAs per SM.  Measured on B200 with a
+    // cold state: 128 units of d = 128 3.27 against 4.78 us per step, 32 units
+    // of d = 64 2.11 against 2.69 us; at 1024 units and more the 256-thread
+    // form is faster.
+    bool big = vec && dk == dv && ((dk == 128 && n_units * 2 <= 2LL * num_sms) || (dk == 64 && n_units <= 2LL * num_sms));
+    if (big) cb = dk / 64;
     if (vec && tuning().decode_col_blocks >= 0) {
         cb = tuning().decode_col_blocks;
         big = false;
