@@ -55,6 +55,26 @@ struct PerDeviceOnce {
     }
 };
 
+// Launch `kern` as a programmatic dependent of the previous kernel in the
+// stream: it may start while that kernel drains, so it must call
+// griddepcontrol.wait before touching global memory the previous kernel
+// writes (every kernel launched this way does).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // Everything a prefill kernel needs to locate its units.  Dense input:
 // groups = B*H, rows_per_group = T, unit u = group u.  Packed input:
 // groups = H, rows_per_group = T_total, unit u = (seq u / H, head u % H).

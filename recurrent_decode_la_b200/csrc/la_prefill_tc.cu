@@ -240,6 +240,11 @@ __global__ void __launch_bounds__(512, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_slot;
+    // Launched as a programmatic dependent of the previous kernel (unsplit
+    // input): the set-up above overlapped its tail; no global memory is
+    // touched before this wait (which returns at once for an ordinary launch).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 #ifdef LINATTN_TRACE
     if (p.trace && threadIdx.x == 0 && blockIdx.x < p.trace_cap / 64) {
         p.trace[62 * (p.trace_cap / 64) + blockIdx.x] = globaltimer_ns();
@@ -1000,6 +1005,9 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_base_slot;
     const uint32_t sbase = smem_u32(smem);
+    // programmatic dependent launch: no global memory before this wait
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1120,8 +1128,8 @@ static cudaError_t launch_sub_impl(const PrefillProblem& p, const CUtensorMap& t
     const int64_t items = p.n_units * p.subs_per_unit;
     const int64_t grid = items < num_sms ? items : num_sms;
     if (grid < 1) return cudaSuccess;
-    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::SMEM, s>>>(tk, tv, p, sub_states);
-    return cudaGetLastError();
+    e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(Cfg::kThreads), Cfg::SMEM, s, tk, tv, p, sub_states);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -1139,23 +1147,35 @@ cudaError_t launch_subsegment_states(const PrefillProblem& p, const CUtensorMap&
 
 // seg_states[u][s] = S_0[u] + sum_{j < s*k} sub_states[u][j] for every segment
 // s (s = 0 is a copy of S_0): one thread per float4 of a unit's state walks
-// the sub-segment sums once, in order.
+// the sub-segment sums once, in order.  The loads go out eight at a time (the
+// additions stay in order, so the sums are the same).
 __global__ void segment_prefix_kernel(const float4* __restrict__ s0, const float4* __restrict__ sub,
                                       float4* __restrict__ seg, int64_t n_units, int d4, int subs_per_seg,
                                       int seg_count) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
     if (i >= n_units * d4) return;
     const int64_t u = i / d4, e = i % d4;
     const int subs = (seg_count - 1) * subs_per_seg;
     float4 acc = s0[u * d4 + e];
     seg[(u * seg_count) * d4 + e] = acc;
-    for (int j = 0; j < subs; ++j) {
-        const float4 x = sub[(u * subs + j) * d4 + e];
-        acc.x += x.x;
-        acc.y += x.y;
-        acc.z += x.z;
-        acc.w += x.w;
-        if ((j + 1) % subs_per_seg == 0) seg[(u * seg_count + (j + 1) / subs_per_seg) * d4 + e] = acc;
+    for (int j0 = 0; j0 < subs; j0 += 8) {
+        float4 x[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+            if (j0 + t < subs) x[t] = sub[(u * subs + j0 + t) * d4 + e];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const int j = j0 + t;
+            if (j < subs) {
+                acc.x += x[t].x;
+                acc.y += x[t].y;
+                acc.z += x[t].z;
+                acc.w += x[t].w;
+                if ((j + 1) % subs_per_seg == 0) seg[(u * seg_count + (j + 1) / subs_per_seg) * d4 + e] = acc;
+            }
+        }
     }
 }
 
@@ -1164,10 +1184,11 @@ cudaError_t launch_segment_prefix(const PrefillProblem& p, float* seg_states, cu
     const int64_t n = p.n_units * d4;
     if (n <= 0) return cudaSuccess;
     const int threads = 256;
-    segment_prefix_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, s>>>(
-        reinterpret_cast<const float4*>(p.state), reinterpret_cast<const float4*>(p.sub_states),
-        reinterpret_cast<float4*>(seg_states), p.n_units, d4, p.subs_per_seg, p.seg_count);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(segment_prefix_kernel, dim3(static_cast<unsigned>((n + threads - 1) / threads)),
+                               dim3(threads), 0, s, reinterpret_cast<const float4*>(p.state),
+                               reinterpret_cast<const float4*>(p.sub_states), reinterpret_cast<float4*>(seg_states),
+                               p.n_units, d4, p.subs_per_seg, p.seg_count);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Rank of every sequence when sorted by decreasing length (ties: lower index
@@ -1210,6 +1231,12 @@ template <int C, int D>
 static cudaError_t launch_tc_impl(const PrefillProblem& p, const CUtensorMap& tq,
                                   const CUtensorMap& tk, const CUtensorMap& tv,
                                   const CUtensorMap& to, int num_sms, cudaStream_t s) {
+    // A CTA of this kernel holds a whole SM's registers, so CTAs launched
+    // early as programmatic dependents would take the SMs from the previous
+    // kernel while they wait.  After the split's prefix kernel (many small
+    // CTAs still to run) the launch is an ordinary one; the grid-dependency
+    // wait in the kernel then returns at once.
+    const bool pdl = p.seg_count == 1;
     using Cfg = TcCfg<C, D>;
     auto kern = prefill_tc_kernel<C, D>;
     // Raise the dynamic shared-memory limit once per device (not inside a
@@ -1221,7 +1248,12 @@ static cudaError_t launch_tc_impl(const PrefillProblem& p, const CUtensorMap& tq
     const int64_t items = p.n_units * p.seg_count;
     int64_t grid = items < num_sms ? items : num_sms;
     if (grid < 1) return cudaSuccess;
-    kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::SMEM, s>>>(tq, tk, tv, to, p);
+    if (pdl) {
+        e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(Cfg::kThreads), Cfg::SMEM, s, tq, tk, tv, to, p);
+        if (e != cudaSuccess) return e;
+    } else {
+        kern<<<static_cast<unsigned>(grid), Cfg::kThreads, Cfg::SMEM, s>>>(tq, tk, tv, to, p);
+    }
     return cudaGetLastError();
 }
 
