@@ -8,10 +8,10 @@
 // memory bandwidth.  The main kernel splits a unit's d_v columns over a few
 // CTAs (o[j] only needs column j of S', so no reduction crosses CTAs); each
 // thread owns four adjacent columns and a strided set of rows, has all of
-// its 128-bit state loads in flight before any arithmetic, updates the rows,
-// stores them back, and keeps a partial q^T S' for its columns; the partials
-// of the rows are summed by warp shuffles, then across warps in shared
-// memory.
+// its 128-bit state loads in flight before any arithmetic, reads the q, k
+// and v entries it needs itself, updates the rows, stores them back, and
+// keeps a partial q^T S' for its columns; the partials of the rows are
+// summed by warp shuffles, then across warps in shared memory.
 #include <cuda_bf16.h>
 
 #include "la_internal.h"
@@ -37,6 +37,27 @@ __device__ __forceinline__ void dec_out<float>(float* p, int64_t i, float x) {
 template <>
 __device__ __forceinline__ void dec_out<__nv_bfloat16>(__nv_bfloat16* p, int64_t i, float x) {
     p[i] = __float2bfloat16_rn(x);
+}
+
+// Four consecutive entries as floats: one vector load when p is aligned for
+// it (always, for d_v a multiple of 4 and a suitably aligned tensor), else
+// four scalar loads.
+template <typename T>
+__device__ __forceinline__ float4 dec_in4(const T* p);
+template <>
+__device__ __forceinline__ float4 dec_in4<float>(const float* p) {
+    if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) return *reinterpret_cast<const float4*>(p);
+    return make_float4(p[0], p[1], p[2], p[3]);
+}
+template <>
+__device__ __forceinline__ float4 dec_in4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    if ((reinterpret_cast<uintptr_t>(p) & 7) == 0) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        return make_float4(a.x, a.y, b.x, b.y);
+    }
+    return make_float4(__bfloat162float(p[0]), __bfloat162float(p[1]), __bfloat162float(p[2]), __bfloat162float(p[3]));
 }
 
 // Bring the 128-byte line holding p into L2 (a hint: no data is returned).
@@ -136,10 +157,7 @@ __global__ void __launch_bounds__(NT, (NT >= 1024 ? 1 : 4))
     decode_cols_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ o,
                        float* __restrict__ state, int64_t n_units, int dk_arg, int dv_arg, int cb_count) {
     extern __shared__ float sm[];
-    float* qs = sm;
-    float* ks = qs + 128;
-    float* vs = ks + 128;
-    float* red = vs + 128;  // [warps][cols of this CTA]
+    float* red = sm;  // [warps][cols of this CTA]
     const int dk = FDK > 0 ? FDK : dk_arg;
     const int dv = FDK > 0 ? FDK : dv_arg;
     const int64_t u = blockIdx.x / cb_count;
@@ -153,14 +171,16 @@ __global__ void __launch_bounds__(NT, (NT >= 1024 ? 1 : 4))
     const int r0 = tid / cols4;
     float4* S = reinterpret_cast<float4*>(state + u * static_cast<int64_t>(dk) * dv + cbeg) + c4;
     const int row4 = dv >> 2;  // float4 per state row
+    const T* qu = q + u * dk;
+    const T* ku = k + u * dk;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int r = r0; r < dk; r += rpp) prefetch_l2(S + r * row4);
     {
         constexpr int kPer = 128 / static_cast<int>(sizeof(T));  // elements per 128-byte line
         const int i = tid * kPer;
         if (i < dk) {
-            prefetch_l2(q + u * dk + i);
-            prefetch_l2(k + u * dk + i);
+            prefetch_l2(qu + i);
+            prefetch_l2(ku + i);
         }
         if (i < ncol) prefetch_l2(v + u * dv + cbeg + i);
     }
@@ -172,31 +192,34 @@ __global__ void __launch_bounds__(NT, (NT >= 1024 ? 1 : 4))
         const int r = r0 + i * rpp;
         if (FDK > 0 || r < dk) sv[i] = S[r * row4];
     }
-    for (int i = tid; i < dk; i += NT) {
-        qs[i] = dec_in<T>(q, u * dk + i);
-        ks[i] = dec_in<T>(k, u * dk + i);
-    }
-    for (int i = tid; i < ncol; i += NT) vs[i] = dec_in<T>(v, u * dv + cbeg + i);
-    __syncthreads();
-    const float4 vv = make_float4(vs[4 * c4], vs[4 * c4 + 1], vs[4 * c4 + 2], vs[4 * c4 + 3]);
+    // each thread reads the q and k entries of its own rows and the v entries
+    // of its own columns itself (the CTA's threads share them through L1), so
+    // no block barrier stands between the loads and the arithmetic
+    const T* vc = v + u * dv + cbeg + 4 * c4;
+    const float4 vv = dec_in4<T>(vc);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (FDK > 0) {
         // fixed form: NR rows per thread cover d_k exactly, one batch
         static_assert(NR * (NT / (FNC / 4)) == FDK, "rows per thread");
+        float qr[NR], kr[NR];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            qr[i] = dec_in<T>(qu, r0 + i * rpp);
+            kr[i] = dec_in<T>(ku, r0 + i * rpp);
+        }
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
             const int r = r0 + i * rpp;
-            const float kr = ks[r], qr = qs[r];
             float4 s4 = sv[i];
-            s4.x = fmaf(kr, vv.x, s4.x);
-            s4.y = fmaf(kr, vv.y, s4.y);
-            s4.z = fmaf(kr, vv.z, s4.z);
-            s4.w = fmaf(kr, vv.w, s4.w);
+            s4.x = fmaf(kr[i], vv.x, s4.x);
+            s4.y = fmaf(kr[i], vv.y, s4.y);
+            s4.z = fmaf(kr[i], vv.z, s4.z);
+            s4.w = fmaf(kr[i], vv.w, s4.w);
             S[r * row4] = s4;
-            acc.x = fmaf(qr, s4.x, acc.x);
-            acc.y = fmaf(qr, s4.y, acc.y);
-            acc.z = fmaf(qr, s4.z, acc.z);
-            acc.w = fmaf(qr, s4.w, acc.w);
+            acc.x = fmaf(qr[i], s4.x, acc.x);
+            acc.y = fmaf(qr[i], s4.y, acc.y);
+            acc.z = fmaf(qr[i], s4.z, acc.z);
+            acc.w = fmaf(qr[i], s4.w, acc.w);
         }
     } else
 #pragma unroll 1
@@ -212,7 +235,7 @@ __global__ void __launch_bounds__(NT, (NT >= 1024 ? 1 : 4))
         for (int i = 0; i < NR; ++i) {
             const int r = r0 + (rb + i) * rpp;
             if (r < dk) {
-                const float kr = ks[r], qr = qs[r];
+                const float kr = dec_in<T>(ku, r), qr = dec_in<T>(qu, r);
                 float4 s4 = sv[i];
                 s4.x = fmaf(kr, vv.x, s4.x);
                 s4.y = fmaf(kr, vv.y, s4.y);
@@ -227,7 +250,7 @@ __global__ void __launch_bounds__(NT, (NT >= 1024 ? 1 : 4))
         }
     }
     // q^T S' over this CTA's rows: first across the lanes of a warp that own
-    // the same columns (shuffles), then across the 8 warps (shared memory).
+    // the same columns (shuffles), then across the warps (shared memory).
     for (int off = cols4; off < 32; off <<= 1) {
         acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
         acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
@@ -293,7 +316,7 @@ static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_units * cb), 1, 1);
     cfg.blockDim = dim3(big ? 1024 : kDecThreads, 1, 1);
-    cfg.dynamicSmemBytes = sizeof(float) * (3 * 128 + (big ? 32 * 64 : 1024));
+    cfg.dynamicSmemBytes = sizeof(float) * (big ? 32 * 64 : 1024);  // row partials [warps][columns]
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
