@@ -349,10 +349,11 @@ static cudaError_t launch_cols(const T* q, const T* k, const T* v, T* o, float* 
     return cudaLaunchKernelEx(&cfg, decode_cols_kernel<T, 4, 0, 0>, q, k, v, o, state, n_units, dk, dv, cb);
 }
 
-// Column blocks per unit: 32 columns per CTA where d_v allows it (each row
-// piece one 128-byte line; measured best on B200 from 128 to 8192 units),
-// more blocks while the grid covers the SMs less than about three times.
-// Every block is a whole number of float4 columns.
+// Column blocks per unit for the 256-thread form: 32 columns per CTA where
+// d_v allows it (each row piece one 128-byte line; the best 256-thread shape
+// measured on B200 from 128 to 8192 units), more blocks while the grid
+// covers the SMs less than about three times.  Every block is a whole number
+// of float4 columns.
 static int decode_col_blocks(int64_t n_units, int num_sms, int dk, int dv) {
     auto ok = [&](int cb) {
         if (cb < 1 || dv % (4 * cb) != 0) return false;
@@ -382,7 +383,8 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     // cold state: 128 units of d = 128 3.27 against 4.78 us per step, 32 units
     // of d = 64 2.11 against 2.69 us; at 1024 units and more the 256-thread
     // form is faster.
-    bool big = vec && dk == dv && ((dk == 128 && n_units * 2 <= 2LL * num_sms) || (dk == 64 && n_units <= 2LL * num_sms));
+    bool big = vec && dk == dv &&
+               ((dk == 128 && n_units * 2 <= 2LL * num_sms) || (dk == 64 && n_units <= 2LL * num_sms));
     if (big) cb = dk / 64;
     if (vec && tuning().decode_col_blocks >= 0) {
         cb = tuning().decode_col_blocks;
