@@ -1,20 +1,28 @@
 // la_prefill_short.cu -- prefill of a few tokens per unit (T <= 16) from a
 // saved state: the multi-token form of decode.
 //
-// With the whole input as one chunk of T tokens that starts from state S
-// (slides "Chunking, causality, and parallel prefill": "Causal triangle",
-// "Incoming and outgoing state"):
-//     o_t = q_t^T S + sum_{j <= t} (q_t . k_j) v_j,    S' = S + sum_t k_t v_t^T
-// Like a decode step, the cost is one read and one write of the fp32 state;
-// the T tokens only add T (d_k + d_v) inputs.  The d_v columns of a unit's
-// state may be split over CB CTAs when there are fewer units than SMs (o_t[j]
-// needs column j only, so there is no reduction across CTAs).  A CTA first
-// puts its whole state tile in flight with asynchronous copies into shared
-// memory (the bytes in flight are then not limited by registers), stages
-// q and k transposed (a row's tokens contiguous) and v, then each thread
-// takes four adjacent columns and a strided set of rows: it accumulates
-// q_t^T S of its columns for every token t in registers and writes the
-// updated rows straight back.  All arithmetic is fp32.
+// The whole input is one chunk of T tokens that starts from state S (slides
+// "Chunking, causality, and parallel prefill": "Causal triangle", "Incoming
+// and outgoing state"), and within it the kernel follows the recurrence
+// itself: with S_t = S + sum_{j <= t} k_j v_j^T,
+//     o_t = q_t^T S_t,    S' = S_T
+// (the same numbers as q_t^T S + sum_{j <= t} (q_t . k_j) v_j, the causal
+// triangle with its diagonal, in exact arithmetic).  Like a decode step, the
+// cost is one read and one write of the fp32 state; the T tokens only add
+// T (d_k + d_v) inputs.  The d_v columns of a unit's state may be split
+// over CB CTAs when there are fewer units than SMs (o_t[j] needs column j
+// only, so there is no reduction across CTAs).
+//
+// One CTA: the token loads are issued first, then the state tile goes in
+// flight with asynchronous copies into shared memory (the bytes in flight
+// are then not limited by registers); q and k are staged transposed (a
+// row's tokens contiguous) and v as is.  Each thread takes four adjacent
+// columns and a strided set of rows, and copies exactly those state
+// elements, in two groups, so that it starts on the first group's rows
+// while the second lands.  For each row it steps through the tokens:
+// S[r] += k_t[r] v_t, then o_t's partial += q_t[r] S[r], and it writes the
+// final row straight back.  The partials of the rows are summed by warp
+// shuffles, then across warps in shared memory.  All arithmetic is fp32.
 #include <cuda_bf16.h>
 
 #include "la_device.cuh"
@@ -57,10 +65,10 @@ __device__ __forceinline__ void fma4(float4& a, float s, const float4& b) {
 
 // Shared memory (floats) of one CTA: the CTA's state tile [d_k][ncol], q
 // and k transposed [d_k][TM] (a row's tokens are contiguous), v [TM][ncol],
-// the causal scores [TM][TM], per-warp partial outputs [warps][TM][ncol].
+// per-warp partial outputs [warps][TM][ncol].
 __host__ __device__ constexpr size_t short_smem_floats(int tm, int dk, int ncol) {
     return static_cast<size_t>(dk) * ncol + 2 * static_cast<size_t>(dk) * tm +
-           static_cast<size_t>(tm) * ((1 + kShortWarps) * ncol + tm);
+           static_cast<size_t>(tm) * (1 + kShortWarps) * ncol;
 }
 
 // Bring the 128-byte line holding p into L2 (a hint: no data is returned).
@@ -75,7 +83,7 @@ __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
 }
 
 template <typename E, int TM>
-__global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const PrefillProblem p, int cb_count) {
+__global__ void __launch_bounds__(kShortThreads, (TM <= 8 ? 2 : 1)) prefill_short_kernel(const PrefillProblem p, int cb_count) {
     extern __shared__ float4 sm4[];
     float* sm = reinterpret_cast<float*>(sm4);
     const int dk = p.dk, dv = p.dv;
@@ -113,8 +121,7 @@ __global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const P
     float* qT = St + dk * ncol;       // [dk][TM]
     float* kT = qT + dk * TM;         // [dk][TM]
     float* vs = kT + dk * TM;         // [TM][ncol]
-    float* qk = vs + TM * ncol;       // [TM][TM]
-    float* red = qk + TM * TM;        // [warps][TM][ncol]
+    float* red = vs + TM * ncol;      // [warps][TM][ncol]
     const int64_t rbase = group * p.rows_per_group + row0;
     const E* Q = static_cast<const E*>(p.q) + rbase * dk;
     const E* K = static_cast<const E*>(p.k) + rbase * dk;
@@ -124,15 +131,11 @@ __global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const P
 
     // Launched as a programmatic dependent of the previous kernel in the
     // stream: nothing is read from global memory before griddepcontrol.wait
-    // returns.  Before it, the CTA only prefetches its state tile and its
-    // tokens into L2 (a hint; L2 is the point of coherence, so a line the
+    // returns.  Before it, the CTA only prefetches its tokens, then its
+    // state tile, into L2 (a hint; L2 is the point of coherence, so a line the
     // previous kernel writes afterwards is still read correctly), which takes
     // the HBM latency off the chain of a sequence of such calls.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    for (int i = tid; i < dk * ((ncol + 31) / 32); i += kShortThreads) {
-        const int r = i / ((ncol + 31) / 32), c = (i % ((ncol + 31) / 32)) * 32;
-        prefetch_l2(Sg + static_cast<int64_t>(r) * dv + c);
-    }
     {
         constexpr int kPer = 128 / static_cast<int>(sizeof(E));  // elements per 128-byte line
         const int nq = len * dk, nv = len * dv;
@@ -142,83 +145,86 @@ __global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const P
         }
         for (int i = tid * kPer; i < nv; i += kShortThreads * kPer) prefetch_l2(V + i);
     }
+    for (int i = tid; i < dk * ((ncol + 31) / 32); i += kShortThreads) {
+        const int r = i / ((ncol + 31) / 32), c = (i % ((ncol + 31) / 32)) * 32;
+        prefetch_l2(Sg + static_cast<int64_t>(r) * dv + c);
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    // the CTA's whole state tile goes in flight first (async copies into
-    // shared memory, no registers held)
-    for (int i = tid; i < dk * cols4; i += kShortThreads) {
-        const int r = i / cols4, c = i % cols4;
-        cp_async16(St + r * ncol + 4 * c, Sg + static_cast<int64_t>(r) * dv + 4 * c);
+    // the token loads first (d_k, d_v <= 128: at most TM / 2 elements of
+    // each per thread), in registers until the state copies are issued
+    constexpr int kPer = (TM * 128 + kShortThreads - 1) / kShortThreads;
+    float qv[kPer], kv[kPer], vt[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int i = tid + j * kShortThreads;
+        qv[j] = i < len * dk ? elem_in<E>(Q, i) : 0.f;
+        kv[j] = i < len * dk ? elem_in<E>(K, i) : 0.f;
+        const int t = i / ncol, c = i % ncol;
+        vt[j] = (i < TM * ncol && t < len) ? elem_in<E>(V, static_cast<int64_t>(t) * dv + cbeg + c) : 0.f;
+    }
+    // then the state: this thread's rows r0, r0 + rpp, ... of columns
+    // 4*c4 .. 4*c4+3 (the elements it updates), the first nh rows in one
+    // group of asynchronous copies and the rest in a second
+    const int nrow = (dk - r0 + rpp - 1) / rpp;
+    const int nh = (nrow + 1) >> 1;
+    for (int i = 0; i < nh; ++i) {
+        const int r = r0 + i * rpp;
+        cp_async16(St + r * ncol + 4 * c4, Sg + static_cast<int64_t>(r) * dv + 4 * c4);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    {
-        // every token load in flight before the first shared-memory store
-        // (d_k, d_v <= 128: at most TM / 2 elements of each per thread)
-        constexpr int kPer = (TM * 128 + kShortThreads - 1) / kShortThreads;
-        float qv[kPer], kv[kPer], vv[kPer];
+    for (int i = nh; i < nrow; ++i) {
+        const int r = r0 + i * rpp;
+        cp_async16(St + r * ncol + 4 * c4, Sg + static_cast<int64_t>(r) * dv + 4 * c4);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int i = tid + j * kShortThreads;
-            qv[j] = i < len * dk ? elem_in<E>(Q, i) : 0.f;
-            kv[j] = i < len * dk ? elem_in<E>(K, i) : 0.f;
-            const int t = i / ncol, c = i % ncol;
-            vv[j] = (i < TM * ncol && t < len) ? elem_in<E>(V, static_cast<int64_t>(t) * dv + cbeg + c) : 0.f;
+    for (int j = 0; j < kPer; ++j) {
+        const int i = tid + j * kShortThreads;
+        if (i < TM * dk) {  // tokens past the end are zero
+            const int t = i / dk, r = i % dk;
+            qT[r * TM + t] = qv[j];
+            kT[r * TM + t] = kv[j];
         }
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int i = tid + j * kShortThreads;
-            if (i < TM * dk) {  // tokens past the end are zero
-                const int t = i / dk, r = i % dk;
-                qT[r * TM + t] = qv[j];
-                kT[r * TM + t] = kv[j];
-            }
-            if (i < TM * ncol) vs[i] = vv[j];
-        }
+        if (i < TM * ncol) vs[i] = vt[j];
     }
     __syncthreads();
-    // causal scores q_t . k_j, j <= t (diagonal kept, the rest exactly 0)
-    for (int i = tid; i < TM * TM; i += kShortThreads) {
-        const int t = i / TM, j = i % TM;
-        float a = 0.f;
-        if (t < len && j <= t)
-            for (int r = 0; r < dk; ++r) a = fmaf(qT[r * TM + t], kT[r * TM + j], a);
-        qk[i] = a;
-    }
+    const int lane = tid & 31, wid = tid >> 5;
     float4 vv[TM];
 #pragma unroll
     for (int t = 0; t < TM; ++t) vv[t] = reinterpret_cast<const float4*>(vs + t * ncol)[c4];
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
-    // state pass: acc[t] += q_t[r] S[r][cols], then S[r] += sum_t k_t[r] v_t
-    // (tokens past the end have q = k = v = 0 and change nothing)
+    // state pass, row by row: for t = 0 .. TM-1, S[r] += k_t[r] v_t, then
+    // acc[t] += q_t[r] S[r] (tokens past the end have q = k = v = 0 and
+    // change nothing); each thread reads only the state elements it copied,
+    // so waiting for its own copies is enough
     float4 acc[TM];
 #pragma unroll
     for (int t = 0; t < TM; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-    for (int r = r0; r < dk; r += rpp) {
+    auto row = [&](int r) {
         float4 s = reinterpret_cast<const float4*>(St + r * ncol)[c4];
         const float4* q4 = reinterpret_cast<const float4*>(qT + r * TM);
         const float4* k4 = reinterpret_cast<const float4*>(kT + r * TM);
 #pragma unroll
         for (int t4 = 0; t4 < TM / 4; ++t4) {
-            const float4 qq = q4[t4];
+            const float4 kk = k4[t4], qq = q4[t4];
+            fma4(s, kk.x, vv[4 * t4 + 0]);
             fma4(acc[4 * t4 + 0], qq.x, s);
+            fma4(s, kk.y, vv[4 * t4 + 1]);
             fma4(acc[4 * t4 + 1], qq.y, s);
+            fma4(s, kk.z, vv[4 * t4 + 2]);
             fma4(acc[4 * t4 + 2], qq.z, s);
+            fma4(s, kk.w, vv[4 * t4 + 3]);
             fma4(acc[4 * t4 + 3], qq.w, s);
         }
-#pragma unroll
-        for (int t4 = 0; t4 < TM / 4; ++t4) {
-            const float4 kk = k4[t4];
-            fma4(s, kk.x, vv[4 * t4 + 0]);
-            fma4(s, kk.y, vv[4 * t4 + 1]);
-            fma4(s, kk.z, vv[4 * t4 + 2]);
-            fma4(s, kk.w, vv[4 * t4 + 3]);
-        }
         reinterpret_cast<float4*>(Sg + static_cast<int64_t>(r) * dv)[c4] = s;
-    }
+    };
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+#pragma unroll 1
+    for (int i = 0; i < nh; ++i) row(r0 + i * rpp);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll 1
+    for (int i = nh; i < nrow; ++i) row(r0 + i * rpp);
     // sum the q_t^T S partials of the rows: lanes that own the same columns
     // (shuffles), then the warps (shared memory)
-    const int lane = tid & 31, wid = tid >> 5;
 #pragma unroll
     for (int t = 0; t < TM; ++t) {
         for (int off = cols4; off < 32; off <<= 1) {
@@ -230,13 +236,12 @@ __global__ void __launch_bounds__(kShortThreads, 1) prefill_short_kernel(const P
         if (lane < cols4) reinterpret_cast<float4*>(red + (wid * TM + t) * ncol)[lane] = acc[t];
     }
     __syncthreads();
-    // o_t = q_t^T S + sum_{j <= t} (q_t . k_j) v_j
+    // o_t = q_t^T S_t: the warps' partials summed
     for (int i = tid; i < len * ncol; i += kShortThreads) {
         const int t = i / ncol, c = i % ncol;
         float sum = 0.f;
 #pragma unroll
         for (int w = 0; w < kShortWarps; ++w) sum += red[(w * TM + t) * ncol + c];
-        for (int j = 0; j <= t; ++j) sum = fmaf(qk[t * TM + j], vs[j * ncol + c], sum);
         elem_out<E>(O, static_cast<int64_t>(t) * dv + cbeg + c, sum);
     }
 }
