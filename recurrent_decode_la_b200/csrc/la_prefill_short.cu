@@ -45,22 +45,43 @@ template <>
 __device__ __forceinline__ float elem_in<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
     return __bfloat162float(p[i]);
 }
+// Four consecutive outputs: one vector store when p is aligned for it, else
+// four scalar stores.
 template <typename E>
-__device__ __forceinline__ void elem_out(E* p, int64_t i, float x);
+__device__ __forceinline__ void elem_out4(E* p, float4 x);
 template <>
-__device__ __forceinline__ void elem_out<float>(float* p, int64_t i, float x) {
-    p[i] = x;
+__device__ __forceinline__ void elem_out4<float>(float* p, float4 x) {
+    if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+        *reinterpret_cast<float4*>(p) = x;
+    } else {
+        p[0] = x.x;
+        p[1] = x.y;
+        p[2] = x.z;
+        p[3] = x.w;
+    }
 }
 template <>
-__device__ __forceinline__ void elem_out<__nv_bfloat16>(__nv_bfloat16* p, int64_t i, float x) {
-    p[i] = __float2bfloat16_rn(x);
+__device__ __forceinline__ void elem_out4<__nv_bfloat16>(__nv_bfloat16* p, float4 x) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y), b = __floats2bfloat162_rn(x.z, x.w);
+    if ((reinterpret_cast<uintptr_t>(p) & 7) == 0) {
+        uint2 raw;
+        raw.x = *reinterpret_cast<const uint32_t*>(&a);
+        raw.y = *reinterpret_cast<const uint32_t*>(&b);
+        *reinterpret_cast<uint2*>(p) = raw;
+    } else {
+        p[0] = a.x;
+        p[1] = a.y;
+        p[2] = b.x;
+        p[3] = b.y;
+    }
 }
 
+// a += s * b, as two paired fp32 FMAs (sm_100)
 __device__ __forceinline__ void fma4(float4& a, float s, const float4& b) {
-    a.x = fmaf(s, b.x, a.x);
-    a.y = fmaf(s, b.y, a.y);
-    a.z = fmaf(s, b.z, a.z);
-    a.w = fmaf(s, b.w, a.w);
+    const float2 ss = make_float2(s, s);
+    const float2 lo = __ffma2_rn(ss, make_float2(b.x, b.y), make_float2(a.x, a.y));
+    const float2 hi = __ffma2_rn(ss, make_float2(b.z, b.w), make_float2(a.z, a.w));
+    a = make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
 // Shared memory (floats) of one CTA: the CTA's state tile [d_k][ncol], q
@@ -131,8 +152,7 @@ __global__ void __launch_bounds__(kShortThreads, (TM <= 8 ? 2 : 1)) prefill_shor
 
     // Launched as a programmatic dependent of the previous kernel in the
     // stream: nothing is read from global memory before griddepcontrol.wait
-    // returns.  Before it, the CTA only prefetches its tokens, then its
-    // state tile, into L2 (a hint; L2 is the point of coherence, so a line the
+    // returns.  Before it, the CTA only prefetches its tokens into L2 (a hint; L2 is the point of coherence, so a line the
     // previous kernel writes afterwards is still read correctly), which takes
     // the HBM latency off the chain of a sequence of such calls.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -144,10 +164,6 @@ __global__ void __launch_bounds__(kShortThreads, (TM <= 8 ? 2 : 1)) prefill_shor
             prefetch_l2(K + i);
         }
         for (int i = tid * kPer; i < nv; i += kShortThreads * kPer) prefetch_l2(V + i);
-    }
-    for (int i = tid; i < dk * ((ncol + 31) / 32); i += kShortThreads) {
-        const int r = i / ((ncol + 31) / 32), c = (i % ((ncol + 31) / 32)) * 32;
-        prefetch_l2(Sg + static_cast<int64_t>(r) * dv + c);
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the token loads first (d_k, d_v <= 128: at most TM / 2 elements of
@@ -236,13 +252,19 @@ __global__ void __launch_bounds__(kShortThreads, (TM <= 8 ? 2 : 1)) prefill_shor
         if (lane < cols4) reinterpret_cast<float4*>(red + (wid * TM + t) * ncol)[lane] = acc[t];
     }
     __syncthreads();
-    // o_t = q_t^T S_t: the warps' partials summed
-    for (int i = tid; i < len * ncol; i += kShortThreads) {
-        const int t = i / ncol, c = i % ncol;
-        float sum = 0.f;
+    // o_t = q_t^T S_t: the warps' partials summed, four columns per thread
+    for (int i = tid; i < len * cols4; i += kShortThreads) {
+        const int t = i / cols4, c = (i % cols4) * 4;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < kShortWarps; ++w) sum += red[(w * TM + t) * ncol + c];
-        elem_out<E>(O, static_cast<int64_t>(t) * dv + cbeg + c, sum);
+        for (int w = 0; w < kShortWarps; ++w) {
+            const float4 x = *reinterpret_cast<const float4*>(red + (w * TM + t) * ncol + c);
+            sum.x += x.x;
+            sum.y += x.y;
+            sum.z += x.z;
+            sum.w += x.w;
+        }
+        elem_out4<E>(O + static_cast<int64_t>(t) * dv + cbeg + c, sum);
     }
 }
 
