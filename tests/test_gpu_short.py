@@ -111,3 +111,51 @@ def test_prefill_then_short_continuation_equals_longer_prefill():
     assert la.la_device_status() == la.LA_OK
     assert nerr(o, O_ref[:, :, T:]) <= BF16_TOL
     assert nerr(S.reshape(S_ref.shape), S_ref) <= BF16_TOL
+
+
+# Many units (768, more than the SMs: one column block per unit, and at
+# d_k <= 64 the 128-thread CTAs).
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (32, 64), (96, 8)])
+@pytest.mark.parametrize("T", [1, 8, 13])
+def test_short_many_units_dense(dtype, dk, dv, T):
+    B, H = 16, 48
+    assert la.la_prefill_kernel(dtype, T, dk, dv) == "short"
+    q, k, v = inputs.random_qkv(T * 7 + dk + 3 * dv, B, H, T, dk, dv, dtype=dtype)
+    S0 = _state(T + 2 * dk, B, H, dk, dv)
+    O_ref, S_ref = ora.recurrent(q, k, v, S0)
+    o, S = gpu_prefill(q, k, v, S0=S0)
+    tol = tol_for(dtype)
+    assert nerr(o, O_ref) <= tol
+    assert nerr(S.reshape(S_ref.shape), S_ref) <= tol
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_short_many_units_packed_too_long_and_empty(d):
+    """Many packed units (800; at d = 64 the 128-thread CTAs): empty
+    sequences keep their state, a sequence longer than the promised
+    max_seqlen is reported and left untouched, the others match the
+    oracle."""
+    H, max_len = 4, 8
+    lens = np.random.default_rng(4).integers(0, max_len + 1, size=200)
+    lens[[0, 50, 199]] = 0
+    lens[77] = 11  # longer than promised
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    T = int(cu[-1])
+    q, k, v = inputs.random_qkv(91, 1, H, T, d, d, dtype=torch.bfloat16)
+    S0 = _state(17, len(lens), H, d, d)
+    O_ref, S_ref = ora.recurrent(q, k, v, S0, cu_seqlens=cu.numpy())
+    o = torch.zeros(1, H, T, d, dtype=torch.bfloat16, device="cuda")
+    st = S0.reshape(-1, d, d).cuda()
+    la.la_prefill(q.cuda(), k.cuda(), v.cuda(), o, st, cu_seqlens=cu.cuda(), max_seqlen=max_len)
+    assert la.la_device_status() == la.LA_ERR_INVALID_ARG
+    st = st.reshape(len(lens), H, d, d).cpu()
+    assert torch.equal(st[77], S0[77])
+    for n in (0, 50, 199):
+        assert torch.equal(st[n], S0[n])
+    a, b = int(cu[77]), int(cu[78])
+    assert torch.count_nonzero(o[0, :, a:b]) == 0
+    keep_units = [n for n in range(len(lens)) if n != 77]
+    assert nerr(st[keep_units], S_ref[keep_units]) <= BF16_TOL
+    keep = np.r_[0:a, b:T]
+    assert nerr(o[0][:, keep].float().cpu(), O_ref[0][:, keep]) <= BF16_TOL
