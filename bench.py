@@ -799,10 +799,17 @@ def chunked_short_comparison(wl, shapes):
 def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h, dk_h, dv_h, world):
     """The same step through the public API with host buffers: pinned host ->
     device copies of every input and device -> host copies of every output,
-    all inside the timed region.  Sequences are independent, so the step is
-    pipelined per sequence on three streams: the copy-in of sequence b+1 and
-    the copy-out of sequence b-1 overlap the prefill of sequence b
-    (la_prefill on that sequence's slices); the decode steps follow."""
+    all inside the timed region.  Two forms are timed:
+
+    - "batch" (the headline `e2e`): every input copied in, one la_prefill
+      over the whole batch (the timed kernel's launch, same units and
+      chunk), the decode steps, then the outputs copied back.  As in a
+      serving loop, the copy-in of step i+1 (its own stream) overlaps the
+      copy-out of step i (another stream); events order every reuse of a
+      buffer, and the copy of o overlaps the decode steps.
+    - "pipelined": sequences are independent, so the copy-in of sequence
+      b+1 and the copy-out of sequence b-1 overlap the prefill of sequence b
+      (la_prefill on that sequence's H units), then the decode steps."""
     B, H, T, d = wl.B, wl.H, wl.T, wl.d
     pins = [x.pin_memory() for x in (q_h, k_h, v_h, dq_h, dk_h, dv_h)]
     o_h = torch.empty_like(pins[2]).pin_memory()
@@ -812,11 +819,56 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
     o = torch.empty_like(dev_bufs[2])
     od = torch.empty_like(dev_bufs[5])
     st = torch.empty(B * H, d, d, dtype=torch.float32, device=dev)
-    nb = la.la_prefill_workspace_size(wl.torch_dtype, 1, H, T, d, d, 0, chunk)
-    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+    nb_seq = la.la_prefill_workspace_size(wl.torch_dtype, 1, H, T, d, d, 0, chunk)
+    ws_seq = torch.empty(nb_seq, dtype=torch.uint8, device=dev) if nb_seq else None
+    nb_all = la.la_prefill_workspace_size(wl.torch_dtype, B, H, T, d, d, 0, chunk)
+    ws_all = torch.empty(nb_all, dtype=torch.uint8, device=dev) if nb_all else None
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-    def step():
+    def decode_and_copy_out():
+        for i in range(dsteps):
+            la.la_decode_step(dev_bufs[3][i], dev_bufs[4][i], dev_bufs[5][i], od[i], st, stream=stream)
+        fin = torch.cuda.Event()
+        fin.record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(fin)
+            od_h.copy_(od, non_blocking=True)
+            st_h.copy_(st, non_blocking=True)
+        stream.wait_stream(s_out)
+
+    carried = {}  # events of the previous batch step
+
+    def step_batch():
+        with torch.cuda.stream(s_in):
+            if "inputs_read" in carried:  # the previous step's kernels are done with the inputs
+                s_in.wait_event(carried["inputs_read"])
+            for i in range(6):
+                dev_bufs[i].copy_(pins[i], non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(s_in)
+        stream.wait_event(copied)
+        if "outputs_read" in carried:  # the previous step's o, od, state are on the host
+            stream.wait_event(carried["outputs_read"])
+        la.la_state_init(st, None, stream=stream)
+        la.la_prefill(dev_bufs[0], dev_bufs[1], dev_bufs[2], o, st, chunk=chunk, workspace=ws_all, stream=stream)
+        pre = torch.cuda.Event()
+        pre.record(stream)
+        for i in range(dsteps):
+            la.la_decode_step(dev_bufs[3][i], dev_bufs[4][i], dev_bufs[5][i], od[i], st, stream=stream)
+        fin = torch.cuda.Event()
+        fin.record(stream)
+        carried["inputs_read"] = fin
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(pre)
+            o_h.copy_(o, non_blocking=True)
+            s_out.wait_event(fin)
+            od_h.copy_(od, non_blocking=True)
+            st_h.copy_(st, non_blocking=True)
+            out = torch.cuda.Event()
+            out.record(s_out)
+        carried["outputs_read"] = out
+
+    def step_pipelined():
         copied = [torch.cuda.Event() for _ in range(B)]
         done = [torch.cuda.Event() for _ in range(B)]
         with torch.cuda.stream(s_in):
@@ -834,41 +886,45 @@ def e2e_run(args, la, torch, dev, stream, wl, chunk, dsteps, q_h, k_h, v_h, dq_h
             sl = slice(b * H, (b + 1) * H)
             la.la_state_init(st[sl], None, stream=stream)
             la.la_prefill(dev_bufs[0][b:b + 1], dev_bufs[1][b:b + 1], dev_bufs[2][b:b + 1], o[b:b + 1], st[sl],
-                          chunk=chunk, workspace=ws, stream=stream)
+                          chunk=chunk, workspace=ws_seq, stream=stream)
             done[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(done[b])
                 o_h[b].copy_(o[b], non_blocking=True)
         stream.wait_event(dec_in)
-        for i in range(dsteps):
-            la.la_decode_step(dev_bufs[3][i], dev_bufs[4][i], dev_bufs[5][i], od[i], st, stream=stream)
-        fin = torch.cuda.Event()
-        fin.record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(fin)
-            od_h.copy_(od, non_blocking=True)
-            st_h.copy_(st, non_blocking=True)
-        stream.wait_stream(s_out)
+        decode_and_copy_out()
 
     n_steps = max(1, min(args.steps, args.e2e_steps))
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            step()
-        stream.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_steps):
-            step()
-        e1.record(stream)
-    stream.synchronize()
-    ms = e0.elapsed_time(e1)
     h2d = sum(x.numel() * x.element_size() for x in pins)
     d2h = o_h.numel() * o_h.element_size() + od_h.numel() * od_h.element_size() + st_h.numel() * 4
     tokens = B * T + B * dsteps
-    return {"value": world * n_steps * tokens / (ms * 1e-3), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / n_steps,
-            "steps": n_steps, "pipelined": "per sequence: copy-in / prefill / copy-out on three streams",
-            "h2d_gbs": h2d / (ms / n_steps * 1e-3) / 1e9}
+
+    def timed(step):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                step()
+            for x in (stream, s_in, s_out):
+                x.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            s_in.wait_event(e0)  # the first copy-in starts inside the timed region
+            for _ in range(n_steps):
+                step()
+            stream.wait_stream(s_in)
+            stream.wait_stream(s_out)  # the last copy-out ends inside it
+            e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1)
+        return {"value": world * n_steps * tokens / (ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / n_steps,
+                "steps": n_steps, "h2d_gbs": h2d / (ms / n_steps * 1e-3) / 1e9}
+
+    res = timed(step_batch)
+    res["form"] = "batch: copy-in, one la_prefill over all units (the timed kernel's launch), decode, copy-out"
+    pipe = timed(step_pipelined)
+    res["pipelined"] = {"value": pipe["value"], "ms_per_step": pipe["ms_per_step"],
+                        "form": "per sequence: copy-in / la_prefill on H units / copy-out on three streams"}
+    return res
 
 
 def run_short_only(args, wl):
