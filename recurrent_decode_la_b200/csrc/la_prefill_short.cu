@@ -250,8 +250,9 @@ __global__ void __launch_bounds__(NT, (TM <= 8 ? 2 : 1) * (kShortThreadsMax / NT
     const E* V = static_cast<const E*>(p.v) + rbase * dv;
     E* O = static_cast<E*>(p.o) + rbase * dv;
     float* Sg = p.state + u * static_cast<int64_t>(dk) * dv + cbeg;
-    // the token loads first (d_k, d_v <= 128: at most TM / 2 elements of
-    // each per thread), in registers until the state copies are issued
+    // the token loads first (d_k, d_v <= 128: at most TM * 128 / NT
+    // elements of each per thread), in registers until the state copies are
+    // issued
     constexpr int kPer = (TM * 128 + NT - 1) / NT;
     float qv[kPer], kv[kPer], vt[kPer];
 #pragma unroll
