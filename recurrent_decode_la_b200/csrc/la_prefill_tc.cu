@@ -668,7 +668,7 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
                 tc_fence_before();
-                fence_proxy_async_smem();
+                if constexpr (!Cfg::PT) fence_proxy_async_smem();  // P went to shared memory
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&bar[Cfg::B_AEMPTY + b]);
