@@ -88,8 +88,9 @@ la_status la_state_init(float* state, const float* src, int64_t n_units,
  *     of few long sequences into segments; the dynamic, longest-first walk
  *     of packed sequences) and gives the same results.
  * Kernels: at most 16 tokens per unit (T, or max_seqlen), d_v a multiple of
- * 4 and a 16-byte aligned state run the few-token kernel: the whole input as
- * one chunk, one pass over the state, fp32 CUDA cores.  Otherwise bf16 with
+ * 4 and a 16-byte aligned state run the few-token kernel: one pass over the
+ * state, each state row stepped through the tokens (the recurrence itself),
+ * fp32 CUDA cores.  Otherwise bf16 with
  * d_k == d_v in {64, 128}, 16-byte aligned q/k/v/o and chunk in
  * {16, 32, 64, 128} run on the tensor cores (TMA + tcgen05, fp32
  * accumulation, fp32 state on chip); everything else with d_k, d_v <= 128
