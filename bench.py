@@ -81,7 +81,7 @@ def load_peaks():
 
 class ClockSampler:
     """Samples the SM clock and the clock-event (throttle) reasons of one GPU
-    every 100 ms through NVML (read-only queries) while the timed region runs."""
+    every 20 ms through NVML (read-only queries) while the timed region runs."""
 
     REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
                "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
@@ -120,7 +120,7 @@ class ClockSampler:
                 self.samples.append((mhz, mask))
             except Exception as e:
                 self.error = repr(e)
-            self._stop.wait(0.1)
+            self._stop.wait(0.02)
 
     def __exit__(self, *a):
         self._stop.set()
